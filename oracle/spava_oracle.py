@@ -1,0 +1,268 @@
+"""fp64 CPU oracle of the Spava / APB-V approximate-attention prefill.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py``, never by the library.  Slow and plain on
+purpose: every step is numpy fp64 in the order the method states it, with
+``np.matmul`` as the only library primitive.
+
+Source pages: "Spava: Accelerating Long-Video Understanding via
+Sequence-Parallelism-aware Approximate Attention", also titled "APB-V: ..."
+(arXiv 2601.21444).  The most detailed are the gist.science technical summaries
+(German and Portuguese twins):
+  * "Methodology", 1. Framework design -- "Context splitting & ZigZag
+    arrangement": the input embeddings are split into an anchor block B_a, a query
+    block B_qr and context blocks B^(h), one per host;
+  * same section, "Approximate attention mechanism": the anchor block is a fixed
+    initial segment; for each host the most essential key-value pairs are picked
+    by query-to-context attention scores and aggregated into passing blocks that
+    later hosts receive; attention runs over the anchor, the local context, the
+    aggregated passing blocks and the query;
+  * 2. System optimisations -- "Fused context and query forward": partial query
+    results are merged through FlashAttention's lse outputs;
+  * "Limitations": on a single GPU the method degenerates to standard
+    FlashAttention (dense causal attention).
+
+The pages give no formula for the score, no constants and no worked example.
+Readings taken where they are silent (each is a parameter of this oracle):
+  R1  score of key j of host h, KV head g: the max, over the last R query rows i
+      of host h with i >= j and over the query heads c of group g, of
+      s_c(i, j) = (q_{i,c} . k_{j,g}) * scale, scale = d^-1/2.  (max over heads:
+      parity unpinned -- no page value fixes sum vs max.)
+  R2  causal inside the probe: probe row i never scores a key j > i.
+  R3  host 0's anchor positions [0, A) are not passing candidates, so no key is
+      attended twice by a later host (parity unpinned -- a plan-level reading).
+  R4  the last host selects nothing (nothing reads its passing blocks).
+  R5  each earlier host contributes its own P keys per KV head; later hosts see
+      h * P passing keys (not re-compressed).
+  R6  the trailing text (query) segment attends densely and causally to every
+      token before it and contributes no scores.
+  R7  ties in selection: larger score first; equal scores -> lower token index;
+      -0.0 equals +0.0.  The P chosen indices are stored in ascending order.
+  R8  GQA: query head c uses KV head c // (hq / hkv) (parity unpinned).
+"""
+
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """uint16 bf16 bit patterns -> exact float64 values."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def host_offsets(host_sizes: Sequence[int]) -> np.ndarray:
+    """Context splitting: off[0] = 0, off[h+1] = off[h] + B_h (context blocks B^(h))."""
+    sizes = np.asarray(host_sizes, dtype=np.int64)
+    if sizes.ndim != 1 or sizes.size == 0 or (sizes <= 0).any():
+        raise ValueError("host sizes must be a non-empty list of positive ints")
+    off = np.zeros(sizes.size + 1, dtype=np.int64)
+    off[1:] = np.cumsum(sizes)
+    return off
+
+
+def host_of_row(off: np.ndarray, i: int) -> int:
+    """Host whose context block holds visual token i."""
+    return int(np.searchsorted(off, i, side="right") - 1)
+
+
+def _groups(hq: int, hkv: int) -> int:
+    if hq % hkv:
+        raise ValueError("hq must be a multiple of hkv")
+    return hq // hkv
+
+
+def probe_scores(q: np.ndarray, k: np.ndarray, off: np.ndarray, probe_r: int,
+                 scale: float) -> np.ndarray:
+    """Query-to-context scores of every visual key (readings R1, R2).
+
+    q [tokens, hq, d], k [tokens, hkv, d] float64; returns float64 [hkv, N].
+    """
+    hq, hkv = q.shape[1], k.shape[1]
+    G = _groups(hq, hkv)
+    H = len(off) - 1
+    N = int(off[-1])
+    scores = np.empty((hkv, N), dtype=np.float64)
+    for h in range(H):
+        a, e = int(off[h]), int(off[h + 1])
+        if probe_r > e - a:
+            raise ValueError("probe_r exceeds a host block")
+        probe_rows = np.arange(e - probe_r, e)
+        keys = np.arange(a, e)
+        visible = probe_rows[:, None] >= keys[None, :]             # [R, B]  (R2)
+        for g in range(hkv):
+            qg = q[e - probe_r:e, g * G:(g + 1) * G, :]              # [R, G, d]
+            s = np.matmul(qg.transpose(1, 0, 2), k[a:e, g, :].T)     # [G, R, B]
+            s = np.where(visible[None], s * scale, -np.inf)
+            scores[g, a:e] = s.max(axis=(0, 1))
+    return scores
+
+
+def select_passing(scores: np.ndarray, off: np.ndarray, anchor: int, passing: int) -> np.ndarray:
+    """Top-P passing keys of each host h < H-1 and KV head (readings R3, R4, R7).
+
+    ``scores`` may be float64 (oracle) or float32 (the GPU's tensor): comparisons run
+    in the array's own precision.  Returns int64 [H-1, hkv, P], ascending per row.
+    """
+    H = len(off) - 1
+    hkv = scores.shape[0]
+    out = np.empty((max(H - 1, 0), hkv, passing), dtype=np.int64)
+    for h in range(H - 1):
+        lo = int(off[h]) + (anchor if h == 0 else 0)
+        hi = int(off[h + 1])
+        if hi - lo < passing:
+            raise ValueError("fewer candidates than passing keys")
+        cand = np.arange(lo, hi)
+        for g in range(hkv):
+            s = scores[g, lo:hi]
+            if np.isnan(s).any():
+                raise ValueError("NaN score")
+            # np.lexsort: last key is primary.  -s ascending == s descending; equal
+            # values (including -0.0 vs +0.0, which compare equal) fall back to the
+            # token index ascending.
+            order = np.lexsort((cand, -s))
+            out[h, g] = np.sort(cand[order[:passing]])
+    return out
+
+
+def key_set(off: np.ndarray, anchor: int, sel: Optional[np.ndarray], g: int, i: int,
+            n_visual: int) -> np.ndarray:
+    """Keys attended by row i through KV head g: anchor | passing of earlier hosts |
+    own block up to i (causal).  Host 0 and text rows: [0, i] (readings R5, R6)."""
+    if i >= n_visual:
+        return np.arange(0, i + 1)
+    h = host_of_row(off, i)
+    if h == 0:
+        return np.arange(0, i + 1)
+    parts = [np.arange(0, anchor)]
+    parts += [np.asarray(sel[hp, g], dtype=np.int64) for hp in range(h)]
+    parts.append(np.arange(int(off[h]), i + 1))
+    return np.concatenate(parts)
+
+
+def _masked_softmax_attend(logits: np.ndarray, visible: np.ndarray, vals: np.ndarray):
+    """Stable softmax over the visible entries of each row; returns (O, lse)."""
+    z = np.where(visible, logits, -np.inf)
+    m = z.max(axis=1, keepdims=True)
+    p = np.where(visible, np.exp(z - m), 0.0)
+    l = p.sum(axis=1, keepdims=True)
+    o = np.matmul(p, vals) / l
+    return o, (m + np.log(l))[:, 0]
+
+
+def approx_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, off: np.ndarray,
+                     anchor: int, sel: Optional[np.ndarray], scale: float,
+                     row_chunk: int = 512):
+    """Approximate attention of every row (host blocks + trailing text rows).
+
+    Host h >= 1 attends to [anchor | passing of hosts < h | own block, causal];
+    host 0 and text rows attend densely and causally.  Returns O float64
+    [tokens, hq, d] and lse float64 [hq, tokens] (natural log).
+    """
+    NT, hq, d = q.shape
+    hkv = k.shape[1]
+    G = _groups(hq, hkv)
+    H = len(off) - 1
+    N = int(off[-1])
+    O = np.empty((NT, hq, d), dtype=np.float64)
+    lse = np.empty((hq, NT), dtype=np.float64)
+    for h in range(H):
+        a, e = int(off[h]), int(off[h + 1])
+        for g in range(hkv):
+            if h == 0:
+                remote = np.zeros(0, dtype=np.int64)
+            else:
+                remote = np.concatenate([np.arange(0, anchor)] +
+                                        [np.asarray(sel[hp, g], dtype=np.int64) for hp in range(h)])
+            for r0 in range(a, e, row_chunk):
+                r1 = min(e, r0 + row_chunk)
+                keys = np.concatenate([remote, np.arange(a, r1)])
+                visible = np.ones((r1 - r0, keys.size), dtype=bool)
+                visible[:, remote.size:] = np.arange(a, r1)[None, :] <= np.arange(r0, r1)[:, None]
+                kk, vv = k[keys, g, :], v[keys, g, :]
+                for c in range(g * G, (g + 1) * G):
+                    logits = np.matmul(q[r0:r1, c, :], kk.T) * scale
+                    O[r0:r1, c], lse[c, r0:r1] = _masked_softmax_attend(logits, visible, vv)
+    for r0 in range(N, NT, row_chunk):
+        r1 = min(NT, r0 + row_chunk)
+        keys = np.arange(0, r1)
+        visible = keys[None, :] <= np.arange(r0, r1)[:, None]
+        for g in range(hkv):
+            kk, vv = k[:r1, g, :], v[:r1, g, :]
+            for c in range(g * G, (g + 1) * G):
+                logits = np.matmul(q[r0:r1, c, :], kk.T) * scale
+                O[r0:r1, c], lse[c, r0:r1] = _masked_softmax_attend(logits, visible, vv)
+    return O, lse
+
+
+def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, off: np.ndarray,
+                   anchor: int, sel: Optional[np.ndarray], scale: float,
+                   rows: Sequence[int], heads: Sequence[int]):
+    """The same attention for chosen (row, head) pairs only, one at a time through
+    ``key_set``.  Used to check full-size runs on a sample of outputs."""
+    hq, hkv = q.shape[1], k.shape[1]
+    G = _groups(hq, hkv)
+    N = int(off[-1])
+    O = np.empty((len(rows), q.shape[2]), dtype=np.float64)
+    L = np.empty(len(rows), dtype=np.float64)
+    for n, (i, c) in enumerate(zip(rows, heads)):
+        g = int(c) // G
+        keys = key_set(off, anchor, sel, g, int(i), N)
+        s = np.matmul(k[keys, g, :], q[int(i), int(c), :]) * scale
+        m = s.max()
+        p = np.exp(s - m)
+        l = p.sum()
+        O[n] = np.matmul(p, v[keys, g, :]) / l
+        L[n] = m + np.log(l)
+    return O, L
+
+
+def dense_causal(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+                 row_chunk: int = 512):
+    """Standard dense causal attention (what one host degenerates to)."""
+    NT, hq, d = q.shape
+    hkv = k.shape[1]
+    G = _groups(hq, hkv)
+    O = np.empty((NT, hq, d), dtype=np.float64)
+    lse = np.empty((hq, NT), dtype=np.float64)
+    for r0 in range(0, NT, row_chunk):
+        r1 = min(NT, r0 + row_chunk)
+        visible = np.arange(r1)[None, :] <= np.arange(r0, r1)[:, None]
+        for c in range(hq):
+            g = c // G
+            logits = np.matmul(q[r0:r1, c, :], k[:r1, g, :].T) * scale
+            O[r0:r1, c], lse[c, r0:r1] = _masked_softmax_attend(logits, visible, v[:r1, g, :])
+    return O, lse
+
+
+def lse_merge(o1: np.ndarray, l1: np.ndarray, o2: np.ndarray, l2: np.ndarray):
+    """Merge two partial attention results over disjoint key sets through their lse
+    (the fused context + query forward): l = log(e^l1 + e^l2),
+    O = e^(l1-l) O1 + e^(l2-l) O2.  o*: [..., d], l*: [...]."""
+    m = np.maximum(l1, l2)
+    l = m + np.log(np.exp(l1 - m) + np.exp(l2 - m))
+    return np.exp(l1 - l)[..., None] * o1 + np.exp(l2 - l)[..., None] * o2, l
+
+
+def prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, host_sizes: Sequence[int],
+            anchor: int, passing: int, probe_r: int, scale: Optional[float] = None,
+            sel: Optional[np.ndarray] = None, rows=None) -> Dict[str, np.ndarray]:
+    """Whole prefill: split -> score -> select -> approximate attention.
+
+    q/k/v are float64 (see ``bf16_bits_to_f64``).  If ``sel`` is given it replaces
+    the oracle's own selection (to re-run attention with another selection).
+    With ``rows=(rows, heads)`` only those outputs are computed.
+    """
+    d = q.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    off = host_offsets(host_sizes)
+    out: Dict[str, np.ndarray] = {"offsets": off}
+    out["scores"] = probe_scores(q, k, off, probe_r, scale)
+    out["sel"] = select_passing(out["scores"], off, anchor, passing) if sel is None else sel
+    if rows is None:
+        out["O"], out["lse"] = approx_attention(q, k, v, off, anchor, out["sel"], scale)
+    else:
+        out["O"], out["lse"] = attention_rows(q, k, v, off, anchor, out["sel"], scale, *rows)
+    return out
