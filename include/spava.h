@@ -1,0 +1,202 @@
+/*
+ * spava.h -- C ABI of the B200 (sm_100a) approximate-attention prefill of
+ * Spava / APB-V ("Accelerating Long-Video Understanding via
+ * Sequence-Parallelism-aware Approximate Attention", arXiv 2601.21444), with all
+ * hosts virtual on one GPU.
+ *
+ * The method (APB-V technical summary, "Methodology", 1. Framework design):
+ * N visual tokens are split into H contiguous context blocks, one per host;
+ * the first A tokens form the anchor block; every host scores its local keys
+ * with query-to-context attention scores and keeps the best P per KV head as
+ * its passing block; host h's queries attend to
+ *     [anchor | passing blocks of hosts 0..h-1 | own block, causal];
+ * a trailing text (query) segment of T tokens attends densely and causally, and
+ * its partial results over the host blocks are merged through their lse
+ * (2. System optimisations, "Fused context and query forward").  One host is
+ * plain dense causal attention ("Limitations").
+ *
+ * Readings where the pages give no formula (plan-level constants):
+ *   score(g, j) = max over the last R query rows i >= j of the host of key j and
+ *                 over the query heads c of KV group g of (q_{i,c} . k_{j,g}) * scale;
+ *   host 0's anchor tokens are not passing candidates;
+ *   selection ties go to the lower token index, -0.0 == +0.0, indices ascending;
+ *   GQA: query head c uses KV head c / (hq / hkv).
+ *
+ * Conventions for every entry point below.
+ *   Layouts   q [N+T][hq][d], k and v [N+T][hkv][d], o [N+T][hq][d]: bf16,
+ *             d contiguous, visual tokens first, then the T text tokens.
+ *             lse [hq][N+T] fp32, natural log.  scores [hkv][N] fp32.
+ *             idx [H-1][hkv][P] int32, token ids ascending per (host, KV head).
+ *             k_pass, v_pass [hkv][H-1][P][d] bf16 (host-major inside a KV head,
+ *             so hosts 0..h-1 of one KV head are one contiguous run).
+ *   Pointers  all tensor pointers are DEVICE pointers owned by the caller, 16-byte
+ *             aligned; the workspace is 256-byte aligned and at least
+ *             spava_workspace_bytes(plan) bytes.  Outputs must not alias inputs.
+ *   Streams   `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *             stream).  Every call only enqueues work: it never synchronises and
+ *             never allocates device memory.  Calls that share one workspace must
+ *             not overlap in time.
+ *   Errors    argument errors are detected on the host before anything is
+ *             enqueued and return SPAVA_ERR_INVALID_ARG / SPAVA_ERR_UNSUPPORTED;
+ *             spava_last_error() gives a one-line reason (thread-local).  Device
+ *             waits inside the kernels are bounded: a wait that runs out sets an
+ *             error word in the workspace and the kernel returns;
+ *             spava_check_device_error() synchronises the stream, reads that word
+ *             and returns SPAVA_ERR_TIMEOUT if it is set (then clears it).
+ */
+#ifndef SPAVA_H_
+#define SPAVA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SPAVA_OK = 0,
+  SPAVA_ERR_INVALID_ARG = 1,  /* bad size, pointer, alignment or combination */
+  SPAVA_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels handle    */
+  SPAVA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed            */
+  SPAVA_ERR_TIMEOUT = 4       /* a bounded device wait ran out                */
+} spava_status;
+
+/* Flags of spava_score_select. */
+#define SPAVA_SCORES_GIVEN 1u /* skip scoring: select from the caller's scores */
+
+/* Opaque host-side plan: sizes, host block offsets and the cost-sorted work lists
+ * of the attention kernel (uploaded once to a small device table owned by the
+ * plan). */
+typedef struct spava_plan spava_plan;
+
+/*
+ * Build a plan (context splitting: APB-V technical summary, 1. Framework design).
+ *   n_visual     N >= 1 visual tokens; n_text T >= 0 trailing text tokens.
+ *   n_hosts      H >= 1 virtual hosts.
+ *   host_sizes   HOST pointer to H block sizes summing to N, or NULL for an equal
+ *                split (then N % H must be 0).  Copied; the caller keeps ownership.
+ *   anchor       A: tokens [0, A) form the anchor block (0 <= A; H > 1 needs
+ *                A + P <= B_0).
+ *   passing      P: passing keys per host and KV head (P <= B_h for h < H-1).
+ *   probe_r      R: probe queries per host, 16 <= R <= min B_h, R % 16 == 0.
+ *   hq, hkv      query / KV heads, hq % hkv == 0, hq / hkv <= 16.
+ *   head_dim     d in {64, 128}.
+ *   softmax_scale  <= 0 selects 1/sqrt(d).
+ * Needs a current CUDA device (it uploads the plan's device table there).
+ * Returns SPAVA_ERR_INVALID_ARG / _UNSUPPORTED before touching the device when the
+ * sizes are not acceptable.  Release with spava_plan_destroy.
+ */
+spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_text,
+                               int32_t n_hosts, const int32_t* host_sizes,
+                               int32_t anchor, int32_t passing, int32_t probe_r,
+                               int32_t hq, int32_t hkv, int32_t head_dim,
+                               float softmax_scale);
+
+/* Free a plan and its device table (synchronises the device first).  NULL is OK. */
+spava_status spava_plan_destroy(spava_plan* plan);
+
+/* Bytes of scratch the calls below need (scores, indices, passing K/V, text
+ * partials, scheduler counters, error word).  0 if plan is NULL. */
+size_t spava_workspace_bytes(const spava_plan* plan);
+
+/* Host block offsets (HOST array of H+1 ints) and work-list statistics, for
+ * callers that want the plan's view of the split.  Returns H, or -1. */
+int32_t spava_plan_offsets(const spava_plan* plan, int32_t* offsets_out /* H+1 or NULL */);
+
+/*
+ * Query-to-context scoring and passing-block selection (APB-V technical summary,
+ * 1. Framework design, "Approximate attention mechanism": passing blocks hold the
+ * most essential key-value pairs, picked by query-to-context attention scores).
+ *   q, k        device bf16, layouts above.
+ *   scores      device fp32 [hkv][N]: written (every host's keys), or read when
+ *               flags & SPAVA_SCORES_GIVEN.
+ *   idx         device int32 [H-1][hkv][P]: the P best candidates of each host
+ *               h < H-1 and KV head, ties to the lower index, ascending.
+ *   flags       0 or SPAVA_SCORES_GIVEN.
+ *   ws          device workspace.
+ */
+spava_status spava_score_select(const spava_plan* plan, const void* q, const void* k,
+                                float* scores, int32_t* idx, uint32_t flags,
+                                void* ws, void* stream);
+
+/*
+ * Passing ("sending passing blocks to later hosts", 2. System optimisations,
+ * "Overlapped communication"): on one GPU every pass is an on-device gather
+ *   k_pass[g][h][j][:] = k[idx[h][g][j]][g][:], and the same for v.
+ *   k, v     device bf16 [N+T][hkv][d];  idx device int32 [H-1][hkv][P].
+ *   k_pass, v_pass  device bf16 [hkv][H-1][P][d].
+ * Indices outside [0, N) are not checked on the device: callers pass the output of
+ * spava_score_select.
+ */
+spava_status spava_gather_passing(const spava_plan* plan, const void* k, const void* v,
+                                  const int32_t* idx, void* k_pass, void* v_pass,
+                                  void* stream);
+
+/*
+ * The whole approximate-attention prefill of one layer: scoring -> selection ->
+ * gather -> one flash-attention pass per host over
+ * [anchor | passing of hosts < h | own block, causal] (tcgen05/TMEM, bf16 in, fp32
+ * accumulation, online softmax) -> text rows as split-KV partials over the host
+ * blocks merged through their lse.
+ *   q, k, v    device bf16 inputs.
+ *   o          device bf16 [N+T][hq][d] output.
+ *   lse        device fp32 [hq][N+T] output (natural log).
+ *   scores_out, idx_out  optional device buffers ([hkv][N] fp32, [H-1][hkv][P]
+ *              int32): when not NULL the run uses them instead of the workspace,
+ *              so the caller can read the scores and the selection back.
+ */
+spava_status spava_attn_prefill(const spava_plan* plan, const void* q, const void* k,
+                                const void* v, void* o, float* lse, float* scores_out,
+                                int32_t* idx_out, void* ws, void* stream);
+
+/*
+ * Dense causal attention over all N+T tokens on the same kernel (the standard
+ * FlashAttention the method degenerates to on one host; the comparison kernel).
+ * Layouts as above.
+ */
+spava_status spava_dense_causal(const spava_plan* plan, const void* q, const void* k,
+                                const void* v, void* o, float* lse, void* ws, void* stream);
+
+/* Synchronise `stream`, read the workspace error word, clear it.  Returns SPAVA_OK,
+ * SPAVA_ERR_TIMEOUT (a bounded device wait ran out) or SPAVA_ERR_CUDA. */
+spava_status spava_check_device_error(const spava_plan* plan, void* ws, void* stream);
+
+/* Testing aid: the next kernel launches of this plan use a device wait limit of
+ * `ns` nanoseconds (0 restores the default of 2 s), and with `stall_producer` != 0
+ * the attention kernel's load warp issues nothing, so every consumer wait runs out
+ * and the kernel returns with SPAVA_ERR_TIMEOUT recorded.  Never faults or hangs. */
+spava_status spava_plan_set_debug(spava_plan* plan, uint64_t wait_limit_ns, int32_t stall_producer);
+
+/*
+ * Kernel timing hook (for benchmarks).  After spava_profile_begin(plan, max_marks)
+ * every entry point of this plan records a CUDA event on its stream before each
+ * kernel it launches and one after the last; spava_profile_read synchronises the
+ * plan's device, writes for each recorded kernel its label (see
+ * spava_kernel_name) and its duration in ms, returns how many it wrote (at most
+ * `max`, -1 on error) and starts a new recording.  Recording stops silently once
+ * max_marks events are used.  spava_profile_end releases the events.
+ */
+spava_status spava_profile_begin(spava_plan* plan, int32_t max_marks);
+int32_t spava_profile_read(spava_plan* plan, int32_t* labels, float* ms, int32_t max);
+spava_status spava_profile_end(spava_plan* plan);
+
+/* Name of a kernel label: 0 score, 1 select, 2 gather, 3 attention (prefill),
+ * 4 lse merge, 5 attention (dense causal). */
+const char* spava_kernel_name(int32_t label);
+
+/* Static text of a status code. */
+const char* spava_status_string(spava_status status);
+
+/* One-line reason for the last non-OK status returned on this thread ("" if none). */
+const char* spava_last_error(void);
+
+/* Kernel launches enqueued by the last successful call on this thread (for
+ * accounting of launches in benchmarks). */
+int32_t spava_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPAVA_H_ */

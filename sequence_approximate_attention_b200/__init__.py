@@ -1,0 +1,241 @@
+"""Spava / APB-V approximate-attention prefill on B200 (sm_100a), all hosts virtual.
+
+A thin Python binding over the C ABI of ``libspava.so`` (include/spava.h): it checks
+tensor dtypes, shapes, devices and contiguity and passes raw device pointers and
+the current CUDA stream.  Every step of the computation runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback, and every entry point raises if the
+library is missing or the call fails.
+
+Layouts: q [N+T, hq, d], k/v [N+T, hkv, d] bf16; o like q; lse [hq, N+T] fp32;
+scores [hkv, N] fp32; idx [H-1, hkv, P] int32; passing K/V [hkv, H-1, P, d] bf16.
+"""
+
+import ctypes
+from typing import Optional, Sequence
+
+import torch
+
+from . import _lib
+from ._lib import SpavaError, load  # noqa: F401
+
+__all__ = ["Plan", "score_select", "gather_passing", "attn_prefill", "dense_causal",
+           "check_device_error", "SpavaError", "load", "last_launch_count"]
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _expect(t: torch.Tensor, name: str, dtype, shape, device) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+class Plan:
+    """Sizes of one prefill layer plus its device-side work lists (spava_plan)."""
+
+    def __init__(self, n_visual: int, n_text: int, n_hosts: int,
+                 host_sizes: Optional[Sequence[int]], anchor: int, passing: int, probe_r: int,
+                 hq: int, hkv: int, head_dim: int, softmax_scale: float = 0.0,
+                 device: Optional[torch.device] = None):
+        self.lib = _lib.load()
+        self.n_visual, self.n_text, self.n_hosts = int(n_visual), int(n_text), int(n_hosts)
+        self.anchor, self.passing, self.probe_r = int(anchor), int(passing), int(probe_r)
+        self.hq, self.hkv, self.head_dim = int(hq), int(hkv), int(head_dim)
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        sizes = None
+        if host_sizes is not None:
+            arr = (ctypes.c_int32 * len(host_sizes))(*[int(x) for x in host_sizes])
+            sizes = ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32))
+        handle = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            st = self.lib.spava_plan_create(ctypes.byref(handle), self.n_visual, self.n_text,
+                                            self.n_hosts, sizes, self.anchor, self.passing,
+                                            self.probe_r, self.hq, self.hkv, self.head_dim,
+                                            ctypes.c_float(softmax_scale))
+        _lib.check(st, "spava_plan_create")
+        self._h = handle
+        self.workspace_bytes = int(self.lib.spava_workspace_bytes(self._h))
+        off = (ctypes.c_int32 * (self.n_hosts + 1))()
+        self.lib.spava_plan_offsets(self._h, off)
+        self.offsets = [int(x) for x in off]
+
+    @property
+    def handle(self):
+        return self._h
+
+    @property
+    def n_total(self) -> int:
+        return self.n_visual + self.n_text
+
+    def new_workspace(self) -> torch.Tensor:
+        return torch.zeros(max(self.workspace_bytes, 256), dtype=torch.uint8, device=self.device)
+
+    def set_debug(self, wait_limit_ns: int = 0, stall_producer: bool = False) -> None:
+        _lib.check(self.lib.spava_plan_set_debug(self._h, int(wait_limit_ns), int(bool(stall_producer))),
+                   "spava_plan_set_debug")
+
+    # kernel timing hook (spava_profile_*)
+    def profile_begin(self, max_marks: int = 4096) -> None:
+        _lib.check(self.lib.spava_profile_begin(self._h, int(max_marks)), "spava_profile_begin")
+
+    def profile_read(self, max_entries: int = 4096):
+        """[(kernel name, ms), ...] of the kernels recorded since the last read."""
+        labels = (ctypes.c_int32 * max_entries)()
+        ms = (ctypes.c_float * max_entries)()
+        n = self.lib.spava_profile_read(self._h, labels, ms, max_entries)
+        if n < 0:
+            raise SpavaError(3, "spava_profile_read", "event query failed")
+        return [(self.lib.spava_kernel_name(labels[i]).decode(), float(ms[i])) for i in range(n)]
+
+    def profile_end(self) -> None:
+        _lib.check(self.lib.spava_profile_end(self._h), "spava_profile_end")
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            _lib.check(self.lib.spava_plan_destroy(self._h), "spava_plan_destroy")
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # shape helpers
+    def qkv_shapes(self):
+        NT = self.n_total
+        return (NT, self.hq, self.head_dim), (NT, self.hkv, self.head_dim)
+
+    def idx_shape(self):
+        return (max(self.n_hosts - 1, 0), self.hkv, self.passing)
+
+    def pass_shape(self):
+        return (self.hkv, max(self.n_hosts - 1, 0), self.passing, self.head_dim)
+
+    def _check_qkv(self, q, k, v=None):
+        qs, ks = self.qkv_shapes()
+        _expect(q, "q", torch.bfloat16, qs, self.device)
+        _expect(k, "k", torch.bfloat16, ks, self.device)
+        if v is not None:
+            _expect(v, "v", torch.bfloat16, ks, self.device)
+
+
+def _ws(plan: Plan, workspace: Optional[torch.Tensor]) -> torch.Tensor:
+    if workspace is None:
+        workspace = plan.new_workspace()
+    if workspace.dtype != torch.uint8 or workspace.numel() < plan.workspace_bytes or \
+            workspace.device != plan.device or workspace.data_ptr() % 256:
+        raise ValueError("workspace: uint8, 256-byte aligned, >= plan.workspace_bytes on the plan's device")
+    return workspace
+
+
+def score_select(plan: Plan, q: Optional[torch.Tensor], k: Optional[torch.Tensor],
+                 scores: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                 scores_given: bool = False, workspace: Optional[torch.Tensor] = None, stream=None):
+    """spava_score_select: probe scores [hkv, N] fp32 and passing indices [H-1, hkv, P]."""
+    dev = plan.device
+    if scores_given:
+        _expect(scores, "scores", torch.float32, (plan.hkv, plan.n_visual), dev)
+    else:
+        plan._check_qkv(q, k)
+        if scores is None:
+            scores = torch.empty((plan.hkv, plan.n_visual), dtype=torch.float32, device=dev)
+        _expect(scores, "scores", torch.float32, (plan.hkv, plan.n_visual), dev)
+    if idx is None:
+        idx = torch.empty(plan.idx_shape(), dtype=torch.int32, device=dev)
+    _expect(idx, "idx", torch.int32, plan.idx_shape(), dev)
+    ws = _ws(plan, workspace)
+    st = plan.lib.spava_score_select(plan.handle, _ptr(q), _ptr(k), _ptr(scores), _ptr(idx),
+                                     _lib.SPAVA_SCORES_GIVEN if scores_given else 0, _ptr(ws),
+                                     _stream(stream))
+    _lib.check(st, "spava_score_select")
+    return scores, idx
+
+
+def gather_passing(plan: Plan, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor,
+                   k_pass: Optional[torch.Tensor] = None, v_pass: Optional[torch.Tensor] = None,
+                   stream=None):
+    """spava_gather_passing: passing K/V [hkv, H-1, P, d] gathered from k/v by idx."""
+    _, ks = plan.qkv_shapes()
+    _expect(k, "k", torch.bfloat16, ks, plan.device)
+    _expect(v, "v", torch.bfloat16, ks, plan.device)
+    _expect(idx, "idx", torch.int32, plan.idx_shape(), plan.device)
+    if k_pass is None:
+        k_pass = torch.empty(plan.pass_shape(), dtype=torch.bfloat16, device=plan.device)
+    if v_pass is None:
+        v_pass = torch.empty(plan.pass_shape(), dtype=torch.bfloat16, device=plan.device)
+    _expect(k_pass, "k_pass", torch.bfloat16, plan.pass_shape(), plan.device)
+    _expect(v_pass, "v_pass", torch.bfloat16, plan.pass_shape(), plan.device)
+    st = plan.lib.spava_gather_passing(plan.handle, _ptr(k), _ptr(v), _ptr(idx), _ptr(k_pass),
+                                       _ptr(v_pass), _stream(stream))
+    _lib.check(st, "spava_gather_passing")
+    return k_pass, v_pass
+
+
+def attn_prefill(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                 o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                 scores_out: Optional[torch.Tensor] = None, idx_out: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """spava_attn_prefill: the whole approximate-attention prefill of one layer.
+
+    Returns (o [N+T, hq, d] bf16, lse [hq, N+T] fp32)."""
+    plan._check_qkv(q, k, v)
+    dev = plan.device
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((plan.hq, plan.n_total), dtype=torch.float32, device=dev)
+    _expect(o, "o", torch.bfloat16, tuple(q.shape), dev)
+    _expect(lse, "lse", torch.float32, (plan.hq, plan.n_total), dev)
+    if scores_out is not None:
+        _expect(scores_out, "scores_out", torch.float32, (plan.hkv, plan.n_visual), dev)
+    if idx_out is not None:
+        _expect(idx_out, "idx_out", torch.int32, plan.idx_shape(), dev)
+    ws = _ws(plan, workspace)
+    st = plan.lib.spava_attn_prefill(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                     _ptr(scores_out), _ptr(idx_out), _ptr(ws), _stream(stream))
+    _lib.check(st, "spava_attn_prefill")
+    return o, lse
+
+
+def dense_causal(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                 o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """spava_dense_causal: dense causal attention over all N+T tokens."""
+    plan._check_qkv(q, k, v)
+    dev = plan.device
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((plan.hq, plan.n_total), dtype=torch.float32, device=dev)
+    _expect(o, "o", torch.bfloat16, tuple(q.shape), dev)
+    _expect(lse, "lse", torch.float32, (plan.hq, plan.n_total), dev)
+    ws = _ws(plan, workspace)
+    st = plan.lib.spava_dense_causal(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                     _ptr(ws), _stream(stream))
+    _lib.check(st, "spava_dense_causal")
+    return o, lse
+
+
+def check_device_error(plan: Plan, workspace: torch.Tensor, stream=None) -> None:
+    """Synchronise and raise SpavaError(SPAVA_ERR_TIMEOUT) if a bounded device wait ran out."""
+    _lib.check(plan.lib.spava_check_device_error(plan.handle, _ptr(workspace), _stream(stream)),
+               "spava_check_device_error")
+
+
+def last_launch_count() -> int:
+    return int(_lib.load().spava_last_launch_count())

@@ -1,0 +1,84 @@
+"""ctypes view of ``libspava.so`` (the C ABI in include/spava.h)."""
+
+import ctypes
+import os
+
+from . import build as _build
+
+c_int32 = ctypes.c_int32
+c_void_p = ctypes.c_void_p
+c_size_t = ctypes.c_size_t
+
+SPAVA_OK = 0
+SPAVA_ERR_INVALID_ARG = 1
+SPAVA_ERR_UNSUPPORTED = 2
+SPAVA_ERR_CUDA = 3
+SPAVA_ERR_TIMEOUT = 4
+SPAVA_SCORES_GIVEN = 1
+
+# name -> (restype, argtypes); the names and order follow include/spava.h.
+SIGNATURES = {
+    "spava_plan_create": (c_int32, [ctypes.POINTER(c_void_p), c_int32, c_int32, c_int32,
+                                    ctypes.POINTER(c_int32), c_int32, c_int32, c_int32,
+                                    c_int32, c_int32, c_int32, ctypes.c_float]),
+    "spava_plan_destroy": (c_int32, [c_void_p]),
+    "spava_workspace_bytes": (c_size_t, [c_void_p]),
+    "spava_plan_offsets": (c_int32, [c_void_p, ctypes.POINTER(c_int32)]),
+    "spava_score_select": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                     ctypes.c_uint32, c_void_p, c_void_p]),
+    "spava_gather_passing": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_void_p]),
+    "spava_attn_prefill": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "spava_dense_causal": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                     c_void_p, c_void_p, c_void_p]),
+    "spava_check_device_error": (c_int32, [c_void_p, c_void_p, c_void_p]),
+    "spava_plan_set_debug": (c_int32, [c_void_p, ctypes.c_uint64, c_int32]),
+    "spava_status_string": (ctypes.c_char_p, [c_int32]),
+    "spava_last_error": (ctypes.c_char_p, []),
+    "spava_last_launch_count": (c_int32, []),
+    "spava_profile_begin": (c_int32, [c_void_p, c_int32]),
+    "spava_profile_read": (c_int32, [c_void_p, ctypes.POINTER(c_int32), ctypes.POINTER(ctypes.c_float),
+                                     c_int32]),
+    "spava_profile_end": (c_int32, [c_void_p]),
+    "spava_kernel_name": (ctypes.c_char_p, [c_int32]),
+}
+
+_LIB = None
+
+
+class SpavaError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {_status_name(status)}: {detail}")
+
+
+def _status_name(s: int) -> str:
+    return {0: "SPAVA_OK", 1: "SPAVA_ERR_INVALID_ARG", 2: "SPAVA_ERR_UNSUPPORTED",
+            3: "SPAVA_ERR_CUDA", 4: "SPAVA_ERR_TIMEOUT"}.get(s, f"status {s}")
+
+
+def load(build_if_missing: bool = True):
+    """Load libspava.so (building it first if it is missing or older than its sources)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = _build.LIB_PATH
+    if build_if_missing and _build.is_stale():
+        _build.build()
+    if not os.path.exists(path):
+        raise ImportError(f"libspava.so is not built ({path}); run "
+                          "python -m sequence_approximate_attention_b200.build")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _LIB = lib
+    return lib
+
+
+def check(status: int, where: str) -> None:
+    if status != SPAVA_OK:
+        detail = load().spava_last_error().decode(errors="replace")
+        raise SpavaError(status, where, detail)

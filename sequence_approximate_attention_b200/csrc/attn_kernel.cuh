@@ -1,0 +1,524 @@
+// Variable-length, multi-segment flash-attention forward for sm_100a
+// (tcgen05 MMA with TMEM accumulators, TMA loads, warp specialisation).
+//
+// One work item = up to 256 query rows (two 128-row Q tiles) of one query head,
+// attending to the concatenation of up to three KV segments.  A segment is a
+// run of rows of K/V (token positions) or of the gathered passing K/V, optionally
+// causal (key position <= query position).  For a host h >= 1 of the
+// approximate-attention prefill the segments are
+//     [anchor rows 0..A) | passing rows of hosts 0..h-1 | own block, causal]
+// (APB-V technical summary, 1. Framework design, "Approximate attention
+// mechanism"); host 0, dense causal attention and text rows use one causal
+// segment, and text rows split over host blocks write fp32 partials with their
+// lse for a later merge (2. System optimisations, "Fused context and query
+// forward").
+//
+// CTA = 384 threads, one per SM, persistent over a cost-sorted item list:
+//   warp 0      TMA producer: Q tiles, then K_j, V_j into a ring of smem stages
+//   warp 1      MMA issuer:   S_i = Q_i K_j^T (SS), O_i += P_i V_j (P from TMEM)
+//   warp 2      TMEM allocator
+//   warps 4-7   softmax of Q tile 0 (TMEM lanes 0..127, one row per thread)
+//   warps 8-11  softmax of Q tile 1
+// TMEM (512 columns): S_0 | S_1 | O_0 | O_1; P_i (bf16) overwrites the first
+// half of S_i after the row has been read.  The MMA order
+//     S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) ...
+// lets one softmax warpgroup work while the tensor core runs the other tile.
+// Online softmax in the exp2 domain with a lazily updated row max: O is only
+// rescaled when the max grows by more than 2^8, which is exact after the final
+// division by the row sum.
+#pragma once
+
+#include "common.cuh"
+
+namespace spava {
+
+enum : int { kSegCausal = 1, kSegPassing = 2 };
+
+struct AttnSeg {
+  int row0;   // first row (token position, or row of the passing buffer)
+  int len;    // rows in the segment (0 = unused)
+  int flags;  // kSegCausal | kSegPassing
+  int pad;
+};
+
+struct AttnItem {
+  int q_row0;    // first query row (token position)
+  int q_rows;    // 1..256 valid query rows
+  int q_head;    // query head
+  int out_slot;  // < 0: final bf16 output; >= 0: fp32 partial slot
+  AttnSeg seg[3];
+};
+static_assert(sizeof(AttnItem) == 64, "AttnItem layout");
+
+struct AttnParams {
+  const AttnItem* items;
+  int n_items;
+  int group;       // hq / hkv
+  int hq;
+  int n_rows_out;  // rows of o and lse (N + T)
+  __nv_bfloat16* o;
+  float* lse;
+  float* o_part;    // [slots][part_rows][hq][D]
+  float* lse_part;  // [slots][hq][part_rows]
+  int part_row0;
+  int part_rows;
+  float scale_log2;  // softmax scale * log2(e)
+  unsigned int* err_word;
+  uint64_t wait_limit_ns;
+  int stall_producer;
+};
+
+template <int D>
+struct AttnShape {
+  static_assert(D == 64 || D == 128, "head_dim");
+  static constexpr int kHalves = D / 64;            // 128-byte column blocks per row
+  static constexpr int kHalfBytes = 128 * 128;      // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kHalves * kHalfBytes;
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+  static constexpr int kSmemBytes = kBarOff + 512 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);
+  static constexpr uint32_t kIdescO = idesc_bf16_f32(128, D, 0, 1);
+  static constexpr int kThreads = 384;
+  __device__ static constexpr uint32_t tmem_s(int i) { return static_cast<uint32_t>(i * 128); }
+  __device__ static constexpr uint32_t tmem_o(int i) { return static_cast<uint32_t>(256 + i * D); }
+};
+
+__device__ __forceinline__ int attn_num_tiles(const AttnItem& it) {
+  return (it.seg[0].len + 127) / 128 + (it.seg[1].len + 127) / 128 + (it.seg[2].len + 127) / 128;
+}
+
+// Segment s of an item, picked with selects so the item stays in registers
+// (dynamic indexing of the array would put it in local memory).
+__device__ __forceinline__ AttnSeg seg_at(const AttnItem& it, int s) {
+  AttnSeg r;
+  r.row0 = s == 0 ? it.seg[0].row0 : (s == 1 ? it.seg[1].row0 : it.seg[2].row0);
+  r.len = s == 0 ? it.seg[0].len : (s == 1 ? it.seg[1].len : it.seg[2].len);
+  r.flags = s == 0 ? it.seg[0].flags : (s == 1 ? it.seg[1].flags : it.seg[2].flags);
+  r.pad = 0;
+  return r;
+}
+
+// Walks the KV tiles of an item in order: segment s, tile t inside it.
+struct TileCursor {
+  int s, t;
+  __device__ __forceinline__ void start(const AttnItem& it) {
+    s = 0;
+    t = 0;
+    settle(it);
+  }
+  __device__ __forceinline__ void settle(const AttnItem& it) {
+    while (s < 3 && seg_at(it, s).len <= t * 128) {
+      ++s;
+      t = 0;
+    }
+  }
+  __device__ __forceinline__ void next(const AttnItem& it) {
+    ++t;
+    settle(it);
+  }
+  __device__ __forceinline__ bool done() const { return s >= 3; }
+};
+
+// Static longest-first schedule: items are sorted by cost (descending); CTA b takes
+// item r*G + b in even rounds and r*G + G-1-b in odd rounds (snake order).
+__device__ __forceinline__ int attn_sched(int r, int b, int G) { return r * G + ((r & 1) ? (G - 1 - b) : b); }
+
+__device__ __forceinline__ AttnItem load_item(const AttnItem* items, int idx) {
+  const int4* src = reinterpret_cast<const int4*>(items + idx);
+  AttnItem it;
+  int4* dst = reinterpret_cast<int4*>(&it);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) dst[k] = __ldg(src + k);
+  return it;
+}
+
+// Wait on a barrier that no timeout or abort may cut short (draining copies in
+// flight before the CTA exits); still bounded.
+__device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    if (mbar_test(bar, parity)) return true;
+    if (global_timer_ns() - t0 > w.limit_ns) {
+      atomicOr(w.err_word, kErrWaitDrain);
+      return false;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKp,
+                    const __grid_constant__ CUtensorMap tmVp, const AttnParams p) {
+  using S = AttnShape<D>;
+  constexpr uint32_t FULL = 0xffffffffu;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + S::kQOff;
+  uint8_t* sKV = smem + S::kKVOff;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;
+  uint64_t* kv_empty = kv_full + S::kStages;
+  uint64_t* s_full = kv_empty + S::kStages;  // [2]
+  uint64_t* p_full = s_full + 2;             // [2]
+  uint64_t* o_full = p_full + 2;             // [2]
+  uint64_t* drain = o_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < S::kStages; ++s) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_empty + s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full + i, 1);
+      mbar_init(p_full + i, 128);
+      mbar_init(o_full + i, 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 2) tmem_alloc(tmem_slot, S::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, p.err_word, p.wait_limit_ns};
+  const int G = gridDim.x, cta = blockIdx.x;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    int ring = 0, m = 0, q_issued = 0;
+    bool ok = true;
+    if (!p.stall_producer) {
+      for (int r = 0; ok; ++r) {
+        const int idx = attn_sched(r, cta, G);
+        if (idx >= p.n_items) break;
+        const AttnItem it = load_item(p.items, idx);
+        const int kvh = it.q_head / p.group;
+        const bool act1 = it.q_rows > 128;
+        if (m > 0) {
+          ok = __all_sync(FULL, mbar_wait(q_empty, (m - 1) & 1, wc, kErrWaitRelease));
+          if (!ok) break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full, (act1 ? 2 : 1) * S::kTileBytes);
+          for (int i = 0; i < (act1 ? 2 : 1); ++i)
+            for (int hh = 0; hh < S::kHalves; ++hh)
+              tma_load_3d(sQ + i * S::kTileBytes + hh * S::kHalfBytes, &tmQ, q_full, hh * 64, it.q_head,
+                          it.q_row0 + i * 128);
+        }
+        __syncwarp();
+        q_issued = m + 1;
+        TileCursor cur;
+        for (cur.start(it); !cur.done() && ok; cur.next(it)) {
+          const AttnSeg sg = seg_at(it, cur.s);
+          const int row = sg.row0 + cur.t * 128;
+          const bool passing = (sg.flags & kSegPassing) != 0;
+          for (int kv = 0; kv < 2; ++kv) {
+            const int slot = ring % S::kStages, use = ring / S::kStages;
+            if (use > 0) {
+              ok = __all_sync(FULL, mbar_wait(kv_empty + slot, (use - 1) & 1, wc, kErrWaitRelease));
+              if (!ok) break;
+            }
+            if (lane == 0) {
+              uint8_t* dst = sKV + slot * S::kTileBytes;
+              mbar_arrive_expect_tx(kv_full + slot, S::kTileBytes);
+              const CUtensorMap* map = passing ? (kv ? &tmVp : &tmKp) : (kv ? &tmV : &tmK);
+              for (int hh = 0; hh < S::kHalves; ++hh) {
+                if (passing)
+                  tma_load_3d(dst + hh * S::kHalfBytes, map, kv_full + slot, hh * 64, row, kvh);
+                else
+                  tma_load_3d(dst + hh * S::kHalfBytes, map, kv_full + slot, hh * 64, kvh, row);
+              }
+            }
+            __syncwarp();
+            ++ring;
+          }
+        }
+        ++m;
+      }
+    }
+    if (!ok) {
+      // Abort: let every copy this warp issued land before the CTA exits.
+      if (lane == 0) {
+        for (int s = 0; s < S::kStages; ++s) {
+          const int uses = ring / S::kStages + (s < ring % S::kStages ? 1 : 0);
+          if (uses > 0) mbar_wait_drain(kv_full + s, (uses - 1) & 1, wc);
+        }
+        if (q_issued > 0) mbar_wait_drain(q_full, (q_issued - 1) & 1, wc);
+      }
+      __syncwarp();
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    int ring = 0, m = 0;
+    uint32_t pc0 = 0, pc1 = 0;
+    bool ok = true, issued_any = false;
+    auto issue_s = [&](int i, int slot) {
+      const uint32_t qa = smem_u32(sQ + i * S::kTileBytes);
+      const uint32_t ka = smem_u32(sKV + slot * S::kTileBytes);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * S::kHalfBytes + (kk & 3) * 32;
+        mma_ss(tmem + S::tmem_s(i), sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), S::kIdescS,
+               kk > 0 ? 1u : 0u);
+      }
+    };
+    auto issue_pv = [&](int i, int slot, bool acc) {
+      const uint32_t va = smem_u32(sKV + slot * S::kTileBytes);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        mma_ts(tmem + S::tmem_o(i), tmem + S::tmem_s(i) + kk * 8, sdesc_sw128(va + kk * 2048, S::kHalfBytes, 1024),
+               S::kIdescO, (acc || kk > 0) ? 1u : 0u);
+      }
+    };
+    for (int r = 0; ok; ++r) {
+      const int idx = attn_sched(r, cta, G);
+      if (idx >= p.n_items) break;
+      const AttnItem it = load_item(p.items, idx);
+      const int nt = attn_num_tiles(it);
+      const bool act1 = it.q_rows > 128;
+      ok = __all_sync(FULL, mbar_wait(q_full, m & 1, wc, kErrWaitLoad));
+      if (!ok) break;
+      int slotK = ring % S::kStages;
+      ok = __all_sync(FULL, mbar_wait(kv_full + slotK, (ring / S::kStages) & 1, wc, kErrWaitLoad));
+      if (!ok) break;
+      ++ring;
+      tc_fence_after();
+      if (lane == 0) {
+        issue_s(0, slotK);
+        mma_commit(s_full + 0);
+        if (act1) {
+          issue_s(1, slotK);
+          mma_commit(s_full + 1);
+        }
+        mma_commit(kv_empty + slotK);
+        if (nt == 1) mma_commit(q_empty);
+      }
+      issued_any = true;
+      __syncwarp();
+      for (int j = 0; j < nt; ++j) {
+        const int slotV = ring % S::kStages;
+        ok = __all_sync(FULL, mbar_wait(kv_full + slotV, (ring / S::kStages) & 1, wc, kErrWaitLoad));
+        if (!ok) break;
+        ++ring;
+        ok = __all_sync(FULL, mbar_wait(p_full + 0, pc0 & 1, wc, kErrWaitSoftmax));
+        ++pc0;
+        if (!ok) break;
+        tc_fence_after();
+        if (lane == 0) {
+          issue_pv(0, slotV, j > 0);
+          if (j == nt - 1) mma_commit(o_full + 0);
+        }
+        __syncwarp();
+        int slotK2 = -1;
+        if (j + 1 < nt) {
+          slotK2 = ring % S::kStages;
+          ok = __all_sync(FULL, mbar_wait(kv_full + slotK2, (ring / S::kStages) & 1, wc, kErrWaitLoad));
+          if (!ok) break;
+          ++ring;
+          tc_fence_after();
+          if (lane == 0) {
+            issue_s(0, slotK2);
+            mma_commit(s_full + 0);
+          }
+          __syncwarp();
+        }
+        if (act1) {
+          ok = __all_sync(FULL, mbar_wait(p_full + 1, pc1 & 1, wc, kErrWaitSoftmax));
+          ++pc1;
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {
+            issue_pv(1, slotV, j > 0);
+            if (j == nt - 1) mma_commit(o_full + 1);
+            if (j + 1 < nt) {
+              issue_s(1, slotK2);
+              mma_commit(s_full + 1);
+            }
+          }
+          __syncwarp();
+        }
+        if (lane == 0) {
+          mma_commit(kv_empty + slotV);
+          if (j + 1 < nt) {
+            mma_commit(kv_empty + slotK2);
+            if (j + 1 == nt - 1) mma_commit(q_empty);
+          }
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      ++m;
+    }
+    if (issued_any) {
+      // Every MMA issued so far must finish before TMEM is released (on the normal
+      // path the softmax warps have already seen them finish; after an abort they
+      // may still be running).
+      if (lane == 0) {
+        mma_commit(drain);
+        mbar_wait_drain(drain, 0, wc);
+      }
+      __syncwarp();
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int i = (warp - 4) >> 2;  // Q tile of this warpgroup
+    const int qd = warp & 3;        // TMEM lane quarter
+    const int row = qd * 32 + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    const float sl2 = p.scale_log2;
+    uint32_t sc = 0, oc = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int idx = attn_sched(r, cta, G);
+      if (idx >= p.n_items) break;
+      const AttnItem it = load_item(p.items, idx);
+      if (i == 1 && it.q_rows <= 128) continue;
+      const int qrow0 = it.q_row0 + i * 128;
+      const int qpos = qrow0 + row;
+      float m_run = -INFINITY, l_run = 0.f;
+      int j = 0;
+      TileCursor cur;
+      for (cur.start(it); !cur.done(); cur.next(it), ++j) {
+        ok = __all_sync(FULL, mbar_wait(s_full + i, sc & 1, wc, kErrWaitMma));
+        ++sc;
+        if (!ok) break;
+        tc_fence_after();
+        const AttnSeg sg = seg_at(it, cur.s);
+        const int kpos0 = sg.row0 + cur.t * 128;
+        const int valid = min(128, sg.len - cur.t * 128);
+        const bool causal = (sg.flags & kSegCausal) != 0;
+        uint32_t sr[128];
+        tmem_ld_x128(tl + S::tmem_s(i), sr);
+        float tmax = -INFINITY;
+        if (valid < 128 || (causal && kpos0 + 127 > qrow0)) {
+          int lim = valid;
+          if (causal) lim = min(lim, qpos - kpos0 + 1);
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            float x = c < lim ? __uint_as_float(sr[c]) : -INFINITY;
+            sr[c] = __float_as_uint(x);
+            tmax = fmaxf(tmax, x);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) tmax = fmaxf(tmax, __uint_as_float(sr[c]));
+        }
+        const float m_tile = tmax * sl2;
+        float alpha = 1.0f;
+        bool rescale = false;
+        if (j == 0) {
+          m_run = m_tile;
+        } else {
+          const bool need = m_tile > m_run + 8.0f;
+          rescale = __any_sync(FULL, need);
+          if (need) {
+            alpha = fast_exp2(m_run - m_tile);
+            m_run = m_tile;
+          }
+        }
+        const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
+        float rs = 0.f;
+        // P = exp2(s * scale_log2 - m) packed to bf16 pairs in place: pair c lands in
+        // sr[c] after sr[2c], sr[2c+1] have been read.
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * c]), sl2, -m_use));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m_use));
+          rs += p0 + p1;
+          sr[c] = pack_bf16x2(p0, p1);
+        }
+        l_run = l_run * alpha + rs;
+        tmem_st_x64(tl + S::tmem_s(i), *reinterpret_cast<uint32_t(*)[64]>(sr));
+        if (rescale) {
+          // O_i holds the sum up to tile j-1 (its MMA finished before S_i(j) did).
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t ov[32];
+            tmem_ld_x32(tl + S::tmem_o(i) + c0, ov);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+            tmem_st_x32(tl + S::tmem_o(i) + c0, ov);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(p_full + i);
+      }
+      if (!ok) break;
+      ok = __all_sync(FULL, mbar_wait(o_full + i, oc & 1, wc, kErrWaitMma));
+      ++oc;
+      if (!ok) break;
+      tc_fence_after();
+      const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
+      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.0f;
+      const bool store = (i * 128 + row) < it.q_rows;
+      const int grow = qpos;
+      if (it.out_slot < 0) {
+        __nv_bfloat16* orow = p.o + (static_cast<size_t>(grow) * p.hq + it.q_head) * D;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t ov[32];
+          tmem_ld_x32(tl + S::tmem_o(i) + c0, ov);
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(ov[8 * v4 + 0]) * inv_l, __uint_as_float(ov[8 * v4 + 1]) * inv_l);
+              w.y = pack_bf16x2(__uint_as_float(ov[8 * v4 + 2]) * inv_l, __uint_as_float(ov[8 * v4 + 3]) * inv_l);
+              w.z = pack_bf16x2(__uint_as_float(ov[8 * v4 + 4]) * inv_l, __uint_as_float(ov[8 * v4 + 5]) * inv_l);
+              w.w = pack_bf16x2(__uint_as_float(ov[8 * v4 + 6]) * inv_l, __uint_as_float(ov[8 * v4 + 7]) * inv_l);
+              dst[v4] = w;
+            }
+          }
+        }
+        if (store) p.lse[static_cast<size_t>(it.q_head) * p.n_rows_out + grow] = (m_use + log2f(l_run)) * 0.69314718055994531f;
+      } else {
+        const int prow = grow - p.part_row0;
+        float* orow = p.o_part + ((static_cast<size_t>(it.out_slot) * p.part_rows + prow) * p.hq + it.q_head) * D;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t ov[32];
+          tmem_ld_x32(tl + S::tmem_o(i) + c0, ov);
+          if (store) {
+            float4* dst = reinterpret_cast<float4*>(orow + c0);
+#pragma unroll
+            for (int v4 = 0; v4 < 8; ++v4)
+              dst[v4] = make_float4(__uint_as_float(ov[4 * v4 + 0]) * inv_l, __uint_as_float(ov[4 * v4 + 1]) * inv_l,
+                                    __uint_as_float(ov[4 * v4 + 2]) * inv_l, __uint_as_float(ov[4 * v4 + 3]) * inv_l);
+          }
+        }
+        if (store)
+          p.lse_part[(static_cast<size_t>(it.out_slot) * p.hq + it.q_head) * p.part_rows + prow] =
+              (m_use + log2f(l_run)) * 0.69314718055994531f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, S::kTmemCols);
+  }
+}
+
+}  // namespace spava

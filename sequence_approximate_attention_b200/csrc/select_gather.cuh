@@ -1,0 +1,190 @@
+// Passing-block selection (top-P per host and KV head), the on-device "pass" of the
+// passing blocks (a gather), and the lse merge of split-KV partials.
+#pragma once
+
+#include "common.cuh"
+
+namespace spava {
+
+// Order-preserving map fp32 -> uint32 (larger float -> larger key).  -0.0 is first
+// made +0.0, so both zeros get the same key.  NaN never reaches here (scores of
+// finite bf16 inputs are finite).
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+  uint32_t b = __float_as_uint(f);
+  if (b == 0x80000000u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Exclusive prefix sum over the block (blockDim.x a multiple of 32, <= 1024).
+// `scratch` holds 33 uint32.  Also returns the block total through *total.
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* scratch, uint32_t* total) {
+  const int lane = lane_id(), warp = warp_id(), nw = blockDim.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = lane < nw ? scratch[lane] : 0u;
+    uint32_t wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    scratch[lane] = wi - w;  // exclusive warp offsets
+    if (lane == 31) scratch[32] = wi;
+  }
+  __syncthreads();
+  const uint32_t res = scratch[warp] + incl - v;
+  *total = scratch[32];
+  __syncthreads();
+  return res;
+}
+
+// One CTA per (host h < H-1, KV head g).  Candidates: [off[h] + (h == 0 ? A : 0),
+// off[h+1]).  Radix select (four 8-bit digits, most significant first) finds the
+// P-th largest key T and how many keys equal to T are taken; a stable compaction in
+// index order then writes the P winners ascending: keys > T, and the lowest-index
+// keys == T.  Result is bit-exact and independent of thread timing.
+__global__ void __launch_bounds__(1024) select_topp_kernel(const float* __restrict__ scores, int n_visual,
+                                                            const int* __restrict__ off, int anchor, int passing,
+                                                            int hkv, int32_t* __restrict__ idx) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t scan_scratch[33];
+  __shared__ uint32_t sh_prefix, sh_k;
+  const int h = blockIdx.x / hkv, g = blockIdx.x % hkv;
+  const int lo = off[h] + (h == 0 ? anchor : 0), hi = off[h + 1];
+  const int n = hi - lo;
+  const float* s = scores + static_cast<size_t>(g) * n_visual + lo;
+  int32_t* out = idx + (static_cast<size_t>(h) * hkv + g) * passing;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  if (passing <= 0) return;
+
+  uint32_t prefix = 0u, pmask = 0u, k = static_cast<uint32_t>(passing);
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int t = tid; t < 256; t += nt) hist[t] = 0u;
+    __syncthreads();
+    for (int j = tid; j < n; j += nt) {
+      const uint32_t u = ordered_key(__ldg(s + j));
+      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 0xFFu], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // lane l owns bins 255-8l .. 248-8l (descending); find the bin holding rank k.
+      uint32_t c[8], sum = 0u;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        c[t] = hist[255 - 8 * tid - t];
+        sum += c[t];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += y;
+      }
+      const uint32_t excl = incl - sum;
+      if (excl < k && k <= incl) {
+        uint32_t acc = excl;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (acc + c[t] >= k) {
+            sh_prefix = prefix | (static_cast<uint32_t>(255 - 8 * tid - t) << shift);
+            sh_k = k - acc;
+            break;
+          }
+          acc += c[t];
+        }
+      }
+    }
+    __syncthreads();
+    prefix = sh_prefix;
+    k = sh_k;
+    pmask |= 0xFFu << shift;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;       // key of the P-th largest score
+  const uint32_t take_eq = k;      // keys equal to T that are selected (lowest index first)
+
+  // Stable compaction: thread t owns keys [t*per, (t+1)*per).
+  const int per = (n + nt - 1) / nt;
+  const int j0 = min(n, tid * per), j1 = min(n, j0 + per);
+  uint32_t cgt = 0u, ceq = 0u;
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t u = ordered_key(__ldg(s + j));
+    cgt += u > T;
+    ceq += u == T;
+  }
+  uint32_t tot;
+  const uint32_t eq_before = block_exclusive_scan(ceq, scan_scratch, &tot);
+  const uint32_t eq_take = eq_before >= take_eq ? 0u : min(ceq, take_eq - eq_before);
+  uint32_t pos = block_exclusive_scan(cgt + eq_take, scan_scratch, &tot);
+  uint32_t eq_seen = eq_before;
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t u = ordered_key(__ldg(s + j));
+    if (u > T) {
+      out[pos++] = lo + j;
+    } else if (u == T) {
+      if (eq_seen < take_eq) out[pos++] = lo + j;
+      ++eq_seen;
+    }
+  }
+}
+
+// k_pass[g][h][j][:] = k[idx[h][g][j]][g][:] (same for v), 16 bytes per thread.
+__global__ void __launch_bounds__(256) gather_passing_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                                              const int32_t* __restrict__ idx, uint4* __restrict__ kp,
+                                                              uint4* __restrict__ vp, int hkv, int hosts_m1,
+                                                              int passing, int chunks_per_row) {
+  const size_t rows_per_g = static_cast<size_t>(hosts_m1) * passing;
+  const size_t total = static_cast<size_t>(hkv) * rows_per_g * chunks_per_row;
+  for (size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t r = t / chunks_per_row;
+    const int ch = static_cast<int>(t - r * chunks_per_row);
+    const int g = static_cast<int>(r / rows_per_g);
+    const size_t rem = r - static_cast<size_t>(g) * rows_per_g;
+    const int h = static_cast<int>(rem / passing);
+    const int j = static_cast<int>(rem - static_cast<size_t>(h) * passing);
+    const int tok = __ldg(idx + (static_cast<size_t>(h) * hkv + g) * passing + j);
+    const size_t src = (static_cast<size_t>(tok) * hkv + g) * chunks_per_row + ch;
+    kp[t] = __ldg(k + src);
+    vp[t] = __ldg(v + src);
+  }
+}
+
+// Merge of split-KV partials through their lse (APB-V technical summary,
+// 2. System optimisations, "Fused context and query forward"):
+//   lse = log sum_k exp(lse_k),  O = sum_k exp(lse_k - lse) O_k.
+// One warp per (text row, head); slots with lse = -inf contribute nothing.
+__global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict__ o_part,
+                                                         const float* __restrict__ lse_part, int n_slots,
+                                                         int part_rows, int hq, int d, int row0, int n_rows_out,
+                                                         __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = lane_id();
+  if (gw >= part_rows * hq) return;
+  const int t = gw / hq, c = gw % hq;
+  float m = -INFINITY;
+  for (int k = 0; k < n_slots; ++k) m = fmaxf(m, __ldg(lse_part + (static_cast<size_t>(k) * hq + c) * part_rows + t));
+  float wsum = 0.f;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};  // d <= 128: lane owns d/32 <= 4 columns
+  const int per = d / 32;
+  for (int k = 0; k < n_slots; ++k) {
+    const float l = __ldg(lse_part + (static_cast<size_t>(k) * hq + c) * part_rows + t);
+    const float w = (l == -INFINITY) ? 0.f : expf(l - m);
+    wsum += w;
+    const float* src = o_part + ((static_cast<size_t>(k) * part_rows + t) * hq + c) * d;
+    for (int e = 0; e < per; ++e) acc[e] += w * __ldg(src + lane + 32 * e);
+  }
+  const float inv = 1.0f / wsum;
+  __nv_bfloat16* dst = o + (static_cast<size_t>(row0 + t) * hq + c) * d;
+  for (int e = 0; e < per; ++e) dst[lane + 32 * e] = __float2bfloat16_rn(acc[e] * inv);
+  if (lane == 0) lse[static_cast<size_t>(c) * n_rows_out + row0 + t] = m + logf(wsum);
+}
+
+}  // namespace spava

@@ -1,0 +1,684 @@
+// Host side of the C ABI declared in include/spava.h: plan (context splitting and
+// the cost-sorted work lists), argument checks, TMA descriptors and launches.
+//
+// Call graph of spava_attn_prefill, all on the caller's stream:
+//   score_kernel      probe scores of hosts 0..H-2 (tensor cores)
+//   select_topp       top-P passing keys per (host, KV head)
+//   gather_passing    passing K/V into one contiguous buffer per KV head
+//   attn_fwd_kernel   one flash-attention pass per host item, text rows as
+//                     split-KV partials over the host blocks
+//   lse_merge         text partials -> final rows
+#include "spava.h"
+
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "attn_kernel.cuh"
+#include "common.cuh"
+#include "score_kernel.cuh"
+#include "select_gather.cuh"
+
+using spava::AttnItem;
+using spava::AttnParams;
+using spava::AttnSeg;
+using spava::ScoreParams;
+
+namespace {
+
+thread_local std::string g_last_error;
+thread_local int g_last_launches = 0;
+
+spava_status fail(spava_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+spava_status ok() {
+  g_last_error.clear();
+  return SPAVA_OK;
+}
+
+#define SPAVA_CUDA(call)                                                                            \
+  do {                                                                                             \
+    cudaError_t e_ = (call);                                                                       \
+    if (e_ != cudaSuccess) return fail(SPAVA_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor map with 128-byte swizzle over a row-major [d2][d1][d0] tensor;
+// d0 is contiguous.  The box is (64, b1, b2); out-of-range rows read as zero.
+spava_status make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b1,
+                      uint32_t b2) {
+  auto fn = encode_fn();
+  if (!fn) return fail(SPAVA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  const cuuint32_t box[3] = {64, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SPAVA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return SPAVA_OK;
+}
+
+}  // namespace
+
+struct spava_plan {
+  int N = 0, T = 0, H = 0, A = 0, P = 0, R = 0, hq = 0, hkv = 0, d = 0;
+  float scale = 0.f;
+  std::vector<int> off;
+  int device = 0, num_sms = 0;
+  // score chunking: Rc probe tokens per MMA N chunk
+  int rc = 0, n_chunks = 0;
+  // device table (owned)
+  void* dtab = nullptr;
+  int* d_off = nullptr;
+  AttnItem* d_items_pre = nullptr;
+  int n_items_pre = 0;
+  AttnItem* d_items_dense = nullptr;
+  int n_items_dense = 0;
+  int4* d_score_pre = nullptr;  // hosts 0..H-2
+  int n_score_pre = 0;
+  int4* d_score_all = nullptr;  // all hosts
+  int n_score_all = 0;
+  // workspace layout
+  size_t ws_err = 0, ws_scores = 0, ws_idx = 0, ws_kp = 0, ws_vp = 0, ws_opart = 0, ws_lpart = 0, ws_total = 0;
+  // debug knobs
+  uint64_t wait_limit_ns = spava::kDefaultWaitLimitNs;
+  int stall_producer = 0;
+  // kernel timing hook: one event per mark, the label of the kernel that follows
+  // it (-1 = end of call) and the call it belongs to
+  mutable std::vector<cudaEvent_t> prof_ev;
+  mutable std::vector<int> prof_label, prof_call;
+  mutable int prof_used = 0, prof_call_id = 0;
+};
+
+namespace {
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+enum KernelLabel { kLabScore = 0, kLabSelect = 1, kLabGather = 2, kLabAttn = 3, kLabMerge = 4, kLabDense = 5 };
+
+void mark(const spava_plan* p, int label, cudaStream_t st) {
+  if (p->prof_used >= static_cast<int>(p->prof_ev.size())) return;
+  if (cudaEventRecord(p->prof_ev[p->prof_used], st) != cudaSuccess) return;
+  p->prof_label[p->prof_used] = label;
+  p->prof_call[p->prof_used] = p->prof_call_id;
+  ++p->prof_used;
+}
+
+int item_cost(const AttnItem& it) {
+  int tiles = 0;
+  for (int s = 0; s < 3; ++s) tiles += ceil_div(it.seg[s].len, 128);
+  return tiles * (it.q_rows > 128 ? 2 : 1);
+}
+
+void sort_by_cost(std::vector<AttnItem>& v) {
+  std::stable_sort(v.begin(), v.end(), [](const AttnItem& a, const AttnItem& b) { return item_cost(a) > item_cost(b); });
+}
+
+AttnItem blank_item(int q_row0, int q_rows, int q_head, int slot) {
+  AttnItem it;
+  std::memset(&it, 0, sizeof(it));
+  it.q_row0 = q_row0;
+  it.q_rows = q_rows;
+  it.q_head = q_head;
+  it.out_slot = slot;
+  return it;
+}
+
+// Work list of the prefill.  Host h's rows go in 256-row items per query head with
+// the KV list [anchor | passing of hosts < h | own block, causal]; text rows (the
+// query block) are split over the host blocks plus their own causal part, each
+// piece writing an fp32 partial with its lse.
+std::vector<AttnItem> build_prefill_items(const spava_plan& p) {
+  std::vector<AttnItem> v;
+  for (int h = 0; h < p.H; ++h) {
+    const int a = p.off[h], e = p.off[h + 1];
+    for (int r0 = a; r0 < e; r0 += 256) {
+      const int rows = std::min(256, e - r0);
+      for (int c = 0; c < p.hq; ++c) {
+        AttnItem it = blank_item(r0, rows, c, -1);
+        int ns = 0;
+        if (h >= 1 && p.A > 0) it.seg[ns++] = AttnSeg{0, p.A, 0, 0};
+        if (h >= 1 && p.P > 0) it.seg[ns++] = AttnSeg{0, h * p.P, spava::kSegPassing, 0};
+        it.seg[ns++] = AttnSeg{a, r0 + rows - a, spava::kSegCausal, 0};
+        v.push_back(it);
+      }
+    }
+  }
+  for (int r0 = p.N; r0 < p.N + p.T; r0 += 256) {
+    const int rows = std::min(256, p.N + p.T - r0);
+    for (int c = 0; c < p.hq; ++c) {
+      for (int k = 0; k <= p.H; ++k) {
+        AttnItem it = blank_item(r0, rows, c, k);
+        if (k < p.H)
+          it.seg[0] = AttnSeg{p.off[k], p.off[k + 1] - p.off[k], 0, 0};
+        else
+          it.seg[0] = AttnSeg{p.N, r0 + rows - p.N, spava::kSegCausal, 0};
+        v.push_back(it);
+      }
+    }
+  }
+  sort_by_cost(v);
+  return v;
+}
+
+std::vector<AttnItem> build_dense_items(const spava_plan& p) {
+  std::vector<AttnItem> v;
+  const int NT = p.N + p.T;
+  for (int r0 = 0; r0 < NT; r0 += 256) {
+    const int rows = std::min(256, NT - r0);
+    for (int c = 0; c < p.hq; ++c) {
+      AttnItem it = blank_item(r0, rows, c, -1);
+      it.seg[0] = AttnSeg{0, r0 + rows, spava::kSegCausal, 0};
+      v.push_back(it);
+    }
+  }
+  sort_by_cost(v);
+  return v;
+}
+
+std::vector<int4> build_score_items(const spava_plan& p, int h_end) {
+  std::vector<int4> v;
+  for (int h = 0; h < h_end; ++h)
+    for (int g = 0; g < p.hkv; ++g)
+      for (int k0 = p.off[h]; k0 < p.off[h + 1]; k0 += 128) v.push_back(make_int4(h, g, k0, p.off[h + 1]));
+  return v;
+}
+
+template <class K>
+spava_status ensure_smem(K kernel, int bytes) {
+  SPAVA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  return SPAVA_OK;
+}
+
+unsigned int* err_word(const spava_plan* p, void* ws) {
+  return reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + p->ws_err);
+}
+
+spava_status check_plan_ws(const spava_plan* p, void* ws) {
+  if (!p) return fail(SPAVA_ERR_INVALID_ARG, "plan is NULL");
+  if (!ws) return fail(SPAVA_ERR_INVALID_ARG, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(SPAVA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  return SPAVA_OK;
+}
+
+// ------------------------------------------------------------------ launches
+template <int D>
+spava_status launch_score(const spava_plan* p, const void* q, const void* k, float* scores, bool all_hosts,
+                          void* ws, cudaStream_t st) {
+  const int n_items = all_hosts ? p->n_score_all : p->n_score_pre;
+  if (n_items == 0) return SPAVA_OK;
+  CUtensorMap tmK, tmQp;
+  spava_status s;
+  if ((s = make_map(&tmK, k, D, p->hkv, p->N + p->T, 1, 128)) != SPAVA_OK) return s;
+  const int G = p->hq / p->hkv;
+  if ((s = make_map(&tmQp, q, D, p->hq, p->N + p->T, G, p->rc)) != SPAVA_OK) return s;
+  ScoreParams sp;
+  sp.items = all_hosts ? p->d_score_all : p->d_score_pre;
+  sp.n_items = n_items;
+  sp.probe_r = p->R;
+  sp.group = G;
+  sp.chunk_tokens = p->rc;
+  sp.n_chunks = p->n_chunks;
+  sp.n_visual = p->N;
+  sp.scale = p->scale;
+  sp.scores = scores;
+  sp.err_word = err_word(p, ws);
+  sp.wait_limit_ns = p->wait_limit_ns;
+  using S = spava::ScoreShape<D>;
+  if ((s = ensure_smem(spava::score_kernel<D>, S::kSmemBytes)) != SPAVA_OK) return s;
+  const int grid = std::min(n_items, p->num_sms);
+  mark(p, kLabScore, st);
+  spava::score_kernel<D><<<grid, 256, S::kSmemBytes, st>>>(tmK, tmQp, sp);
+  SPAVA_CUDA(cudaGetLastError());
+  ++g_last_launches;
+  return SPAVA_OK;
+}
+
+spava_status launch_select(const spava_plan* p, const float* scores, int32_t* idx, cudaStream_t st) {
+  if (p->H < 2 || p->P == 0) return SPAVA_OK;
+  mark(p, kLabSelect, st);
+  spava::select_topp_kernel<<<(p->H - 1) * p->hkv, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, p->hkv, idx);
+  SPAVA_CUDA(cudaGetLastError());
+  ++g_last_launches;
+  return SPAVA_OK;
+}
+
+spava_status launch_gather(const spava_plan* p, const void* k, const void* v, const int32_t* idx, void* kp, void* vp,
+                           cudaStream_t st) {
+  if (p->H < 2 || p->P == 0) return SPAVA_OK;
+  const int chunks = p->d * 2 / 16;
+  const size_t total = static_cast<size_t>(p->hkv) * (p->H - 1) * p->P * chunks;
+  const int grid = static_cast<int>(std::min<size_t>((total + 255) / 256, static_cast<size_t>(p->num_sms) * 8));
+  mark(p, kLabGather, st);
+  spava::gather_passing_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), idx,
+                                                      static_cast<uint4*>(kp), static_cast<uint4*>(vp), p->hkv,
+                                                      p->H - 1, p->P, chunks);
+  SPAVA_CUDA(cudaGetLastError());
+  ++g_last_launches;
+  return SPAVA_OK;
+}
+
+template <int D>
+spava_status launch_attn(const spava_plan* p, const AttnItem* items, int n_items, const void* q, const void* k,
+                         const void* v, const void* kp, const void* vp, void* o, float* lse, void* ws,
+                         cudaStream_t st) {
+  if (n_items == 0) return SPAVA_OK;
+  CUtensorMap tmQ, tmK, tmV, tmKp, tmVp;
+  spava_status s;
+  const uint64_t NT = static_cast<uint64_t>(p->N) + p->T;
+  if ((s = make_map(&tmQ, q, D, p->hq, NT, 1, 128)) != SPAVA_OK) return s;
+  if ((s = make_map(&tmK, k, D, p->hkv, NT, 1, 128)) != SPAVA_OK) return s;
+  if ((s = make_map(&tmV, v, D, p->hkv, NT, 1, 128)) != SPAVA_OK) return s;
+  if (p->H >= 2 && p->P > 0 && kp && vp) {
+    const uint64_t rows = static_cast<uint64_t>(p->H - 1) * p->P;
+    if ((s = make_map(&tmKp, kp, D, rows, p->hkv, 128, 1)) != SPAVA_OK) return s;
+    if ((s = make_map(&tmVp, vp, D, rows, p->hkv, 128, 1)) != SPAVA_OK) return s;
+  } else {
+    tmKp = tmK;  // never read: no item has a passing segment
+    tmVp = tmV;
+  }
+  AttnParams ap;
+  ap.items = items;
+  ap.n_items = n_items;
+  ap.group = p->hq / p->hkv;
+  ap.hq = p->hq;
+  ap.n_rows_out = p->N + p->T;
+  ap.o = static_cast<__nv_bfloat16*>(o);
+  ap.lse = lse;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  ap.o_part = reinterpret_cast<float*>(w + p->ws_opart);
+  ap.lse_part = reinterpret_cast<float*>(w + p->ws_lpart);
+  ap.part_row0 = p->N;
+  ap.part_rows = p->T;
+  ap.scale_log2 = p->scale * 1.4426950408889634f;
+  ap.err_word = err_word(p, ws);
+  ap.wait_limit_ns = p->wait_limit_ns;
+  ap.stall_producer = p->stall_producer;
+  using S = spava::AttnShape<D>;
+  if ((s = ensure_smem(spava::attn_fwd_kernel<D>, S::kSmemBytes)) != SPAVA_OK) return s;
+  const int grid = std::min(n_items, p->num_sms);
+  mark(p, items == p->d_items_dense ? kLabDense : kLabAttn, st);
+  spava::attn_fwd_kernel<D><<<grid, S::kThreads, S::kSmemBytes, st>>>(tmQ, tmK, tmV, tmKp, tmVp, ap);
+  SPAVA_CUDA(cudaGetLastError());
+  ++g_last_launches;
+  return SPAVA_OK;
+}
+
+spava_status launch_merge(const spava_plan* p, void* o, float* lse, void* ws, cudaStream_t st) {
+  if (p->T == 0) return SPAVA_OK;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const int warps = p->T * p->hq;
+  const int grid = (warps * 32 + 255) / 256;
+  mark(p, kLabMerge, st);
+  spava::lse_merge_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(w + p->ws_opart),
+                                                 reinterpret_cast<const float*>(w + p->ws_lpart), p->H + 1, p->T,
+                                                 p->hq, p->d, p->N, p->N + p->T, static_cast<__nv_bfloat16*>(o), lse);
+  SPAVA_CUDA(cudaGetLastError());
+  ++g_last_launches;
+  return SPAVA_OK;
+}
+
+spava_status begin_call(const spava_plan* p, void* ws, cudaStream_t st) {
+  g_last_launches = 0;
+  ++p->prof_call_id;
+  int dev = -1;
+  SPAVA_CUDA(cudaGetDevice(&dev));
+  if (dev != p->device) return fail(SPAVA_ERR_INVALID_ARG, "current device %d differs from the plan's device %d", dev, p->device);
+  SPAVA_CUDA(cudaMemsetAsync(err_word(p, ws), 0, 256, st));
+  return SPAVA_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+const char* spava_status_string(spava_status s) {
+  switch (s) {
+    case SPAVA_OK: return "SPAVA_OK";
+    case SPAVA_ERR_INVALID_ARG: return "SPAVA_ERR_INVALID_ARG";
+    case SPAVA_ERR_UNSUPPORTED: return "SPAVA_ERR_UNSUPPORTED";
+    case SPAVA_ERR_CUDA: return "SPAVA_ERR_CUDA";
+    case SPAVA_ERR_TIMEOUT: return "SPAVA_ERR_TIMEOUT";
+  }
+  return "SPAVA_ERR_UNKNOWN";
+}
+
+const char* spava_last_error(void) { return g_last_error.c_str(); }
+
+int32_t spava_last_launch_count(void) { return g_last_launches; }
+
+spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_text, int32_t n_hosts,
+                               const int32_t* host_sizes, int32_t anchor, int32_t passing, int32_t probe_r,
+                               int32_t hq, int32_t hkv, int32_t head_dim, float softmax_scale) {
+  if (!out) return fail(SPAVA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (n_visual < 1 || n_text < 0 || n_hosts < 1) return fail(SPAVA_ERR_INVALID_ARG, "need N >= 1, T >= 0, H >= 1");
+  if (n_hosts > n_visual) return fail(SPAVA_ERR_INVALID_ARG, "more hosts than visual tokens");
+  if (hq < 1 || hkv < 1 || hq % hkv) return fail(SPAVA_ERR_INVALID_ARG, "hq must be a positive multiple of hkv");
+  if (hq / hkv > 16) return fail(SPAVA_ERR_UNSUPPORTED, "query heads per KV head must be <= 16");
+  if (head_dim != 64 && head_dim != 128) return fail(SPAVA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (anchor < 0 || passing < 0 || probe_r < 0) return fail(SPAVA_ERR_INVALID_ARG, "negative A, P or R");
+  if (static_cast<int64_t>(n_visual) + n_text > (1ll << 30))
+    return fail(SPAVA_ERR_UNSUPPORTED, "more than 2^30 tokens");
+  std::vector<int> off(n_hosts + 1, 0);
+  if (host_sizes) {
+    int64_t sum = 0;
+    for (int h = 0; h < n_hosts; ++h) {
+      if (host_sizes[h] < 1) return fail(SPAVA_ERR_INVALID_ARG, "host %d has size %d", h, host_sizes[h]);
+      sum += host_sizes[h];
+      off[h + 1] = static_cast<int>(sum);
+    }
+    if (sum != n_visual) return fail(SPAVA_ERR_INVALID_ARG, "host sizes sum to %lld, not N=%d", (long long)sum, n_visual);
+  } else {
+    if (n_visual % n_hosts) return fail(SPAVA_ERR_INVALID_ARG, "equal split needs N %% H == 0");
+    for (int h = 0; h < n_hosts; ++h) off[h + 1] = off[h] + n_visual / n_hosts;
+  }
+  int min_b = n_visual;
+  for (int h = 0; h < n_hosts; ++h) min_b = std::min(min_b, off[h + 1] - off[h]);
+  if (n_hosts > 1) {
+    if (probe_r < 1 || probe_r > min_b) return fail(SPAVA_ERR_INVALID_ARG, "need 1 <= R <= min block size (%d)", min_b);
+    if (probe_r % 16) return fail(SPAVA_ERR_UNSUPPORTED, "R must be a multiple of 16");
+    if (anchor + passing > off[1]) return fail(SPAVA_ERR_INVALID_ARG, "host 0 needs A + P <= B_0");
+    for (int h = 1; h < n_hosts - 1; ++h)
+      if (passing > off[h + 1] - off[h]) return fail(SPAVA_ERR_INVALID_ARG, "P exceeds block %d", h);
+  }
+  if (anchor > n_visual) return fail(SPAVA_ERR_INVALID_ARG, "A > N");
+
+  spava_plan* p = new spava_plan();
+  p->N = n_visual;
+  p->T = n_text;
+  p->H = n_hosts;
+  p->A = anchor;
+  p->P = passing;
+  p->R = probe_r;
+  p->hq = hq;
+  p->hkv = hkv;
+  p->d = head_dim;
+  p->scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  p->off = off;
+  const int G = hq / hkv;
+  p->rc = std::max(16, 16 * (256 / (16 * G)));
+  if (probe_r > 0) p->rc = std::min(p->rc, probe_r);
+  p->n_chunks = probe_r > 0 ? ceil_div(probe_r, p->rc) : 0;
+
+  // workspace layout
+  size_t o = 0;
+  p->ws_err = o;
+  o += 256;
+  p->ws_scores = o;
+  o = align_up(o + static_cast<size_t>(hkv) * n_visual * 4, 256);
+  const size_t hm1 = n_hosts > 1 ? n_hosts - 1 : 0;
+  p->ws_idx = o;
+  o = align_up(o + hm1 * hkv * passing * 4, 256);
+  p->ws_kp = o;
+  o = align_up(o + hm1 * hkv * passing * head_dim * 2, 256);
+  p->ws_vp = o;
+  o = align_up(o + hm1 * hkv * passing * head_dim * 2, 256);
+  p->ws_opart = o;
+  o = align_up(o + static_cast<size_t>(n_hosts + 1) * n_text * hq * head_dim * 4, 256);
+  p->ws_lpart = o;
+  o = align_up(o + static_cast<size_t>(n_hosts + 1) * hq * n_text * 4, 256);
+  p->ws_total = o;
+
+  // device
+  auto bail = [&](spava_status s) {
+    if (p->dtab) cudaFree(p->dtab);
+    delete p;
+    return s;
+  };
+  cudaError_t e = cudaGetDevice(&p->device);
+  if (e != cudaSuccess) return bail(fail(SPAVA_ERR_CUDA, "no CUDA device: %s", cudaGetErrorString(e)));
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, p->device);
+  if (e != cudaSuccess) return bail(fail(SPAVA_ERR_CUDA, "cudaGetDeviceProperties: %s", cudaGetErrorString(e)));
+  if (prop.major != 10 || prop.minor != 0)
+    return bail(fail(SPAVA_ERR_UNSUPPORTED, "needs an sm_100 (B200) device, found sm_%d%d", prop.major, prop.minor));
+  p->num_sms = prop.multiProcessorCount;
+
+  const auto pre = build_prefill_items(*p);
+  const auto dense = build_dense_items(*p);
+  const auto sc_pre = build_score_items(*p, n_hosts - 1);
+  const auto sc_all = build_score_items(*p, n_hosts);
+  p->n_items_pre = static_cast<int>(pre.size());
+  p->n_items_dense = static_cast<int>(dense.size());
+  p->n_score_pre = static_cast<int>(sc_pre.size());
+  p->n_score_all = static_cast<int>(sc_all.size());
+  const size_t b_off = align_up(off.size() * 4, 256);
+  const size_t b_pre = align_up(pre.size() * sizeof(AttnItem), 256);
+  const size_t b_dense = align_up(dense.size() * sizeof(AttnItem), 256);
+  const size_t b_spre = align_up(sc_pre.size() * sizeof(int4), 256);
+  const size_t b_sall = align_up(sc_all.size() * sizeof(int4), 256);
+  std::vector<uint8_t> host(b_off + b_pre + b_dense + b_spre + b_sall, 0);
+  size_t at = 0;
+  std::memcpy(host.data() + at, off.data(), off.size() * 4);
+  at += b_off;
+  if (!pre.empty()) std::memcpy(host.data() + at, pre.data(), pre.size() * sizeof(AttnItem));
+  at += b_pre;
+  if (!dense.empty()) std::memcpy(host.data() + at, dense.data(), dense.size() * sizeof(AttnItem));
+  at += b_dense;
+  if (!sc_pre.empty()) std::memcpy(host.data() + at, sc_pre.data(), sc_pre.size() * sizeof(int4));
+  at += b_spre;
+  if (!sc_all.empty()) std::memcpy(host.data() + at, sc_all.data(), sc_all.size() * sizeof(int4));
+  e = cudaMalloc(&p->dtab, host.size());
+  if (e != cudaSuccess) return bail(fail(SPAVA_ERR_CUDA, "cudaMalloc(plan table): %s", cudaGetErrorString(e)));
+  e = cudaMemcpy(p->dtab, host.data(), host.size(), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return bail(fail(SPAVA_ERR_CUDA, "cudaMemcpy(plan table): %s", cudaGetErrorString(e)));
+  uint8_t* base = static_cast<uint8_t*>(p->dtab);
+  p->d_off = reinterpret_cast<int*>(base);
+  p->d_items_pre = reinterpret_cast<AttnItem*>(base + b_off);
+  p->d_items_dense = reinterpret_cast<AttnItem*>(base + b_off + b_pre);
+  p->d_score_pre = reinterpret_cast<int4*>(base + b_off + b_pre + b_dense);
+  p->d_score_all = reinterpret_cast<int4*>(base + b_off + b_pre + b_dense + b_spre);
+  *out = p;
+  return ok();
+}
+
+spava_status spava_plan_destroy(spava_plan* p) {
+  if (!p) return ok();
+  spava_status s = SPAVA_OK;
+  for (cudaEvent_t e : p->prof_ev) cudaEventDestroy(e);
+  if (p->dtab) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaFree(p->dtab);
+    if (e != cudaSuccess) s = fail(SPAVA_ERR_CUDA, "plan destroy: %s", cudaGetErrorString(e));
+  }
+  delete p;
+  return s == SPAVA_OK ? ok() : s;
+}
+
+size_t spava_workspace_bytes(const spava_plan* p) { return p ? p->ws_total : 0; }
+
+int32_t spava_plan_offsets(const spava_plan* p, int32_t* offsets_out) {
+  if (!p) return -1;
+  if (offsets_out)
+    for (int h = 0; h <= p->H; ++h) offsets_out[h] = p->off[h];
+  return p->H;
+}
+
+spava_status spava_plan_set_debug(spava_plan* p, uint64_t wait_limit_ns, int32_t stall_producer) {
+  if (!p) return fail(SPAVA_ERR_INVALID_ARG, "plan is NULL");
+  p->wait_limit_ns = wait_limit_ns ? wait_limit_ns : spava::kDefaultWaitLimitNs;
+  p->stall_producer = stall_producer ? 1 : 0;
+  return ok();
+}
+
+spava_status spava_score_select(const spava_plan* p, const void* q, const void* k, float* scores, int32_t* idx,
+                                uint32_t flags, void* ws, void* stream) {
+  spava_status s;
+  if ((s = check_plan_ws(p, ws)) != SPAVA_OK) return s;
+  if (!scores || !idx) return fail(SPAVA_ERR_INVALID_ARG, "scores and idx must not be NULL");
+  if (!(flags & SPAVA_SCORES_GIVEN) && (!q || !k)) return fail(SPAVA_ERR_INVALID_ARG, "q and k must not be NULL");
+  if (!(flags & SPAVA_SCORES_GIVEN) && (!aligned16(q) || !aligned16(k)))
+    return fail(SPAVA_ERR_INVALID_ARG, "q and k must be 16-byte aligned");
+  if (flags & ~SPAVA_SCORES_GIVEN) return fail(SPAVA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = begin_call(p, ws, st)) != SPAVA_OK) return s;
+  if (!(flags & SPAVA_SCORES_GIVEN) && p->H >= 1) {
+    if (p->R == 0) return fail(SPAVA_ERR_INVALID_ARG, "plan has R = 0: nothing to score");
+    s = p->d == 128 ? launch_score<128>(p, q, k, scores, true, ws, st) : launch_score<64>(p, q, k, scores, true, ws, st);
+    if (s != SPAVA_OK) return s;
+  }
+  if ((s = launch_select(p, scores, idx, st)) != SPAVA_OK) return s;
+  mark(p, -1, st);
+  return ok();
+}
+
+spava_status spava_gather_passing(const spava_plan* p, const void* k, const void* v, const int32_t* idx, void* k_pass,
+                                  void* v_pass, void* stream) {
+  if (!p) return fail(SPAVA_ERR_INVALID_ARG, "plan is NULL");
+  if (!k || !v || !idx || !k_pass || !v_pass) return fail(SPAVA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_pass) || !aligned16(v_pass))
+    return fail(SPAVA_ERR_INVALID_ARG, "k, v, k_pass, v_pass must be 16-byte aligned");
+  g_last_launches = 0;
+  ++p->prof_call_id;
+  spava_status s = launch_gather(p, k, v, idx, k_pass, v_pass, static_cast<cudaStream_t>(stream));
+  if (s != SPAVA_OK) return s;
+  mark(p, -1, static_cast<cudaStream_t>(stream));
+  return ok();
+}
+
+spava_status spava_attn_prefill(const spava_plan* p, const void* q, const void* k, const void* v, void* o, float* lse,
+                                float* scores_out, int32_t* idx_out, void* ws, void* stream) {
+  spava_status s;
+  if ((s = check_plan_ws(p, ws)) != SPAVA_OK) return s;
+  if (!q || !k || !v || !o || !lse) return fail(SPAVA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(SPAVA_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = begin_call(p, ws, st)) != SPAVA_OK) return s;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* scores = scores_out ? scores_out : reinterpret_cast<float*>(w + p->ws_scores);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + p->ws_idx);
+  void* kp = w + p->ws_kp;
+  void* vp = w + p->ws_vp;
+  if (p->H >= 2 && p->P > 0) {
+    s = p->d == 128 ? launch_score<128>(p, q, k, scores, false, ws, st) : launch_score<64>(p, q, k, scores, false, ws, st);
+    if (s != SPAVA_OK) return s;
+    if ((s = launch_select(p, scores, idx, st)) != SPAVA_OK) return s;
+    if ((s = launch_gather(p, k, v, idx, kp, vp, st)) != SPAVA_OK) return s;
+  }
+  s = p->d == 128 ? launch_attn<128>(p, p->d_items_pre, p->n_items_pre, q, k, v, kp, vp, o, lse, ws, st)
+                  : launch_attn<64>(p, p->d_items_pre, p->n_items_pre, q, k, v, kp, vp, o, lse, ws, st);
+  if (s != SPAVA_OK) return s;
+  if ((s = launch_merge(p, o, lse, ws, st)) != SPAVA_OK) return s;
+  mark(p, -1, st);
+  return ok();
+}
+
+spava_status spava_dense_causal(const spava_plan* p, const void* q, const void* k, const void* v, void* o, float* lse,
+                                void* ws, void* stream) {
+  spava_status s;
+  if ((s = check_plan_ws(p, ws)) != SPAVA_OK) return s;
+  if (!q || !k || !v || !o || !lse) return fail(SPAVA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(SPAVA_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = begin_call(p, ws, st)) != SPAVA_OK) return s;
+  s = p->d == 128 ? launch_attn<128>(p, p->d_items_dense, p->n_items_dense, q, k, v, nullptr, nullptr, o, lse, ws, st)
+                  : launch_attn<64>(p, p->d_items_dense, p->n_items_dense, q, k, v, nullptr, nullptr, o, lse, ws, st);
+  if (s != SPAVA_OK) return s;
+  mark(p, -1, st);
+  return ok();
+}
+
+spava_status spava_profile_begin(spava_plan* p, int32_t max_marks) {
+  if (!p || max_marks < 2) return fail(SPAVA_ERR_INVALID_ARG, "need a plan and max_marks >= 2");
+  spava_profile_end(p);
+  p->prof_ev.assign(max_marks, nullptr);
+  for (auto& e : p->prof_ev) SPAVA_CUDA(cudaEventCreate(&e));
+  p->prof_label.assign(max_marks, -1);
+  p->prof_call.assign(max_marks, -1);
+  p->prof_used = 0;
+  return ok();
+}
+
+int32_t spava_profile_read(spava_plan* p, int32_t* labels, float* ms, int32_t max) {
+  if (!p) return -1;
+  if (p->prof_used > 0 && cudaEventSynchronize(p->prof_ev[p->prof_used - 1]) != cudaSuccess) return -1;
+  int n = 0;
+  for (int k = 0; k + 1 < p->prof_used && n < max; ++k) {
+    if (p->prof_label[k] < 0 || p->prof_call[k] != p->prof_call[k + 1]) continue;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, p->prof_ev[k], p->prof_ev[k + 1]) != cudaSuccess) return -1;
+    if (labels) labels[n] = p->prof_label[k];
+    if (ms) ms[n] = t;
+    ++n;
+  }
+  p->prof_used = 0;
+  return n;
+}
+
+spava_status spava_profile_end(spava_plan* p) {
+  if (!p) return fail(SPAVA_ERR_INVALID_ARG, "plan is NULL");
+  if (!p->prof_ev.empty()) cudaDeviceSynchronize();
+  for (cudaEvent_t e : p->prof_ev)
+    if (e) cudaEventDestroy(e);
+  p->prof_ev.clear();
+  p->prof_label.clear();
+  p->prof_call.clear();
+  p->prof_used = 0;
+  return ok();
+}
+
+const char* spava_kernel_name(int32_t label) {
+  switch (label) {
+    case kLabScore: return "score";
+    case kLabSelect: return "select";
+    case kLabGather: return "gather";
+    case kLabAttn: return "attention";
+    case kLabMerge: return "lse_merge";
+    case kLabDense: return "attention_dense";
+  }
+  return "unknown";
+}
+
+spava_status spava_check_device_error(const spava_plan* p, void* ws, void* stream) {
+  spava_status s;
+  if ((s = check_plan_ws(p, ws)) != SPAVA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SPAVA_CUDA(cudaStreamSynchronize(st));
+  unsigned int word = 0;
+  SPAVA_CUDA(cudaMemcpy(&word, err_word(p, ws), sizeof(word), cudaMemcpyDeviceToHost));
+  if (word) {
+    SPAVA_CUDA(cudaMemsetAsync(err_word(p, ws), 0, 256, st));
+    SPAVA_CUDA(cudaStreamSynchronize(st));
+    return fail(SPAVA_ERR_TIMEOUT, "a bounded device wait ran out (error bits 0x%x)", word);
+  }
+  return ok();
+}
+
+}  // extern "C"

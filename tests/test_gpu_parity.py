@@ -1,0 +1,227 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle, on small
+shapes that span several tiles, ragged tails and the method's degenerate cases.
+
+Acceptance (per the workload definition):
+  * selection bit-exact against the oracle's selection run on the GPU's fp32 scores;
+  * against the fp64 oracle scores, selections may differ only at near-ties
+    (P-th vs (P+1)-th score closer than 1e-4);
+  * O within 2e-2 and lse within 1e-3 of the oracle re-run with the GPU's indices;
+  * scores within 1e-5 * scale * sum|q k| (fp32 accumulation of exact bf16 products).
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import spava_oracle as orc
+from workloads import CONFIGS, generate
+
+from .helpers import (check_selection_vs_fp64, compare_attention, inputs, make_plan, score_tolerance,
+                      to_device_bf16)
+
+pytestmark = pytest.mark.gpu
+
+sab = pytest.importorskip("sequence_approximate_attention_b200")
+
+TINY = CONFIGS["tiny"]
+
+# name -> (workload, explicit host sizes or None)
+CASES = {
+    "tiny": (TINY, None),
+    "tiny_h1": (TINY.with_(n_hosts=1), None),
+    "tiny_h4_text1": (TINY.with_(n_hosts=4, n_text=1), None),
+    "tiny_h8": (TINY.with_(n_hosts=8, anchor=16, passing=16, probe_r=16), None),
+    "tiny_text128": (TINY.with_(n_text=128), None),
+    "tiny_text300": (TINY.with_(n_text=300), None),
+    "tiny_no_anchor_no_passing": (TINY.with_(anchor=0, passing=0, n_text=40), None),
+    "tiny_p1": (TINY.with_(passing=1, anchor=5), None),
+    "tiny_pmax": (TINY.with_(n_hosts=4, anchor=0, passing=128, n_text=9), None),
+    "d128_g7_uneven": (TINY.with_(n_visual=1024, n_hosts=4, head_dim=128, hq=14, hkv=2, anchor=64,
+                                  passing=64, probe_r=32, n_text=77, kv_kind="frame", frame=64,
+                                  salient_frac=0.05, seed=7), [192, 320, 256, 256]),
+    "d128_ragged": (TINY.with_(n_visual=512, n_hosts=2, head_dim=128, hq=8, hkv=2, anchor=8, passing=40,
+                               probe_r=16, n_text=5, seed=8), [200, 312]),
+    "d128_g16_r128": (TINY.with_(n_visual=768, n_hosts=3, head_dim=128, hq=16, hkv=1, anchor=32,
+                                 passing=96, probe_r=128, n_text=0, seed=9), None),
+}
+
+
+def _sizes(cfg, sizes):
+    if sizes is not None:
+        return np.asarray(sizes, dtype=np.int32)
+    return generate(cfg)["host_sizes"]
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_prefill_matches_oracle(name):
+    cfg, sizes = CASES[name]
+    cfg = cfg.with_(uneven=None)
+    g, f64, dev = inputs(cfg)
+    sizes = _sizes(cfg, sizes)
+    plan = make_plan(sab, cfg, sizes)
+    off = orc.host_offsets(sizes)
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    ws = plan.new_workspace()
+    scores = torch.full((cfg.hkv, cfg.n_visual), float("nan"), device="cuda")
+    idx = torch.full(plan.idx_shape(), -1, dtype=torch.int32, device="cuda")
+    o, lse = sab.attn_prefill(plan, dev["q"], dev["k"], dev["v"], scores_out=scores, idx_out=idx,
+                              workspace=ws)
+    sab.check_device_error(plan, ws)
+    torch.cuda.synchronize()
+    H = cfg.n_hosts
+    sel = idx.cpu().numpy().astype(np.int64)
+    if H > 1 and cfg.passing > 0:
+        sc = scores.cpu().numpy()
+        n_sc = int(off[H - 1])
+        ref_scores = orc.probe_scores(f64["q"], f64["k"], off, cfg.probe_r, scale)
+        tol = score_tolerance(f64["q"], f64["k"], off, cfg.probe_r, scale)
+        err = np.abs(sc[:, :n_sc] - ref_scores[:, :n_sc])
+        assert (err <= tol[:, :n_sc]).all(), f"score error {err.max()}"
+        # bit-exact selection on the GPU's own fp32 scores
+        np.testing.assert_array_equal(sel, orc.select_passing(sc, off, cfg.anchor, cfg.passing))
+        check_selection_vs_fp64(sel, ref_scores, off, cfg.anchor, cfg.passing)
+    O_ref, L_ref = orc.approx_attention(f64["q"], f64["k"], f64["v"], off, cfg.anchor,
+                                        sel if H > 1 else None, scale)
+    compare_attention(o, lse, O_ref, L_ref, name)
+    plan.close()
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_text300", "d128_g7_uneven"])
+def test_dense_causal_matches_oracle(name):
+    cfg, sizes = CASES[name]
+    g, f64, dev = inputs(cfg.with_(uneven=None))
+    plan = make_plan(sab, cfg, _sizes(cfg, sizes))
+    ws = plan.new_workspace()
+    o, lse = sab.dense_causal(plan, dev["q"], dev["k"], dev["v"], workspace=ws)
+    sab.check_device_error(plan, ws)
+    O_ref, L_ref = orc.dense_causal(f64["q"], f64["k"], f64["v"], 1.0 / math.sqrt(cfg.head_dim))
+    compare_attention(o, lse, O_ref, L_ref, "dense " + name)
+    plan.close()
+
+
+def test_one_host_prefill_equals_dense_kernel():
+    cfg = TINY.with_(n_hosts=1, n_text=33)
+    g, f64, dev = inputs(cfg)
+    plan = make_plan(sab, cfg, [cfg.n_visual])
+    o1, l1 = sab.attn_prefill(plan, dev["q"], dev["k"], dev["v"])
+    o2, l2 = sab.dense_causal(plan, dev["q"], dev["k"], dev["v"])
+    torch.cuda.synchronize()
+    assert (o1.float() - o2.float()).abs().max().item() <= 2e-2
+    assert (l1 - l2).abs().max().item() <= 1e-3
+
+
+@pytest.mark.parametrize("name", ["tiny", "d128_g7_uneven", "d128_g16_r128"])
+def test_score_select_all_hosts(name):
+    cfg, sizes = CASES[name]
+    g, f64, dev = inputs(cfg.with_(uneven=None))
+    sizes = _sizes(cfg, sizes)
+    plan = make_plan(sab, cfg, sizes)
+    off = orc.host_offsets(sizes)
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    scores, idx = sab.score_select(plan, dev["q"], dev["k"])
+    torch.cuda.synchronize()
+    sc = scores.cpu().numpy()
+    ref = orc.probe_scores(f64["q"], f64["k"], off, cfg.probe_r, scale)
+    tol = score_tolerance(f64["q"], f64["k"], off, cfg.probe_r, scale)
+    assert (np.abs(sc - ref) <= tol).all()
+    np.testing.assert_array_equal(idx.cpu().numpy(), orc.select_passing(sc, off, cfg.anchor, cfg.passing))
+    plan.close()
+
+
+def _adversarial_scores(rng, hkv, N):
+    s = rng.integers(-4, 5, size=(hkv, N)).astype(np.float32)   # heavy exact ties
+    s[0, ::7] = -0.0
+    s[0, 3::7] = 0.0
+    if hkv > 1:
+        s[1] = 2.5                                               # all equal
+    if hkv > 2:
+        s[2] = rng.standard_normal(N).astype(np.float32) * np.float32(1e30)
+        s[2, 100:110] = np.float32(3.0e38)
+        s[2, 200:210] = np.float32(-3.0e38)
+    if hkv > 3:
+        s[3] = np.float32(1.0) + np.arange(N, dtype=np.float32) * np.float32(1e-7)  # near-equal ramp
+    return s
+
+
+@pytest.mark.parametrize("sizes,anchor,passing", [
+    ([8192] * 3, 1024, 1024), ([4096, 12288, 6144, 9216], 2048, 2048), ([300, 500, 224], 10, 290),
+    ([64, 64], 0, 64), ([1000, 24], 0, 1)])
+def test_select_bit_exact_with_ties(sizes, anchor, passing):
+    rng = np.random.default_rng(len(sizes) * 100 + passing)
+    hkv = 4
+    N = int(sum(sizes))
+    cfg = TINY.with_(n_visual=N, n_hosts=len(sizes), anchor=anchor, passing=passing, probe_r=16,
+                     hq=4, hkv=hkv, head_dim=64)
+    plan = make_plan(sab, cfg, sizes)
+    s = _adversarial_scores(rng, hkv, N)
+    scores = torch.from_numpy(s).cuda()
+    _, idx = sab.score_select(plan, None, None, scores=scores, scores_given=True)
+    torch.cuda.synchronize()
+    off = orc.host_offsets(sizes)
+    np.testing.assert_array_equal(idx.cpu().numpy(), orc.select_passing(s, off, anchor, passing))
+    plan.close()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_gather_byte_exact(d):
+    cfg = TINY.with_(n_visual=2048, n_hosts=4, head_dim=d, hq=8, hkv=4, anchor=16, passing=100, n_text=3)
+    g = generate(cfg)
+    plan = make_plan(sab, cfg, g["host_sizes"])
+    k, v = to_device_bf16(g["k"]), to_device_bf16(g["v"])
+    rng = np.random.default_rng(0)
+    idx_np = np.sort(rng.integers(0, cfg.n_visual, size=plan.idx_shape()), axis=-1).astype(np.int32)
+    kp, vp = sab.gather_passing(plan, k, v, torch.from_numpy(idx_np).cuda())
+    torch.cuda.synchronize()
+    kb, vb = g["k"], g["v"]
+    want_k = np.empty(plan.pass_shape(), dtype=np.uint16)
+    want_v = np.empty(plan.pass_shape(), dtype=np.uint16)
+    for h in range(cfg.n_hosts - 1):
+        for gg in range(cfg.hkv):
+            want_k[gg, h] = kb[idx_np[h, gg], gg]
+            want_v[gg, h] = vb[idx_np[h, gg], gg]
+    np.testing.assert_array_equal(kp.view(torch.int16).cpu().numpy().view(np.uint16), want_k)
+    np.testing.assert_array_equal(vp.view(torch.int16).cpu().numpy().view(np.uint16), want_v)
+    plan.close()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """With the load warp told to issue nothing, every wait runs out after 20 ms: the
+    call reports SPAVA_ERR_TIMEOUT, and the same plan then runs correctly."""
+    cfg = TINY.with_(n_text=20)
+    g, f64, dev = inputs(cfg)
+    plan = make_plan(sab, cfg, g["host_sizes"])
+    ws = plan.new_workspace()
+    plan.set_debug(wait_limit_ns=20_000_000, stall_producer=True)
+    sab.attn_prefill(plan, dev["q"], dev["k"], dev["v"], workspace=ws)
+    with pytest.raises(sab.SpavaError) as ei:
+        sab.check_device_error(plan, ws)
+    assert ei.value.status == 4
+    plan.set_debug(0, False)
+    idx = torch.empty(plan.idx_shape(), dtype=torch.int32, device="cuda")
+    o, lse = sab.attn_prefill(plan, dev["q"], dev["k"], dev["v"], idx_out=idx, workspace=ws)
+    sab.check_device_error(plan, ws)
+    off = orc.host_offsets(g["host_sizes"])
+    O_ref, L_ref = orc.approx_attention(f64["q"], f64["k"], f64["v"], off, cfg.anchor,
+                                        idx.cpu().numpy().astype(np.int64), 1 / math.sqrt(cfg.head_dim))
+    compare_attention(o, lse, O_ref, L_ref, "after timeout")
+    plan.close()
+
+
+def test_bad_arguments_raise_before_launch():
+    cfg = TINY
+    g, f64, dev = inputs(cfg)
+    plan = make_plan(sab, cfg, g["host_sizes"])
+    with pytest.raises(ValueError):
+        sab.attn_prefill(plan, dev["q"][:-1], dev["k"], dev["v"])
+    with pytest.raises(TypeError):
+        sab.attn_prefill(plan, dev["q"].float(), dev["k"], dev["v"])
+    lib = plan.lib
+    ws = plan.new_workspace()
+    import ctypes
+    st = lib.spava_attn_prefill(plan.handle, ctypes.c_void_p(dev["q"].data_ptr() + 2), ctypes.c_void_p(dev["k"].data_ptr()),
+                                ctypes.c_void_p(dev["v"].data_ptr()), ctypes.c_void_p(dev["q"].data_ptr()),
+                                ctypes.c_void_p(ws.data_ptr()), None, None, ctypes.c_void_p(ws.data_ptr()), None)
+    assert st == 1  # misaligned q
+    plan.close()
