@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Benchmark of the approximate-attention prefill (one layer) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 128k] [--impl b200|reference]
+
+A step is one call of spava_attn_prefill over the whole hot path (probe scoring,
+top-P selection, passing gather, the attention pass, the text lse merge) on one
+seeded synthetic layer whose inputs already sit in HBM.  Q/K/V of the default
+workload (2.1 GB + 2 x 0.27 GB) are far larger than the 126 MB L2, so no flush is
+needed between steps.  With N GPUs (torchrun, NCCL) every rank runs its own replica
+of the workload (weak scaling, no data-path collective); the time is the max over
+ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (rank 0 only),
+each step a bounded sample of the same workload.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import CONFIGS, generate  # noqa: E402
+
+METRIC = "approx-attn prefill tokens/s and % of B200 BF16 tensor peak at 128K tokens"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- workload arithmetic
+def attended_pairs(cfg, sizes):
+    """(query, key) pairs the approximate attention evaluates (per query head)."""
+    N, T, A, P = cfg.n_visual, cfg.n_text, cfg.anchor, cfg.passing
+    pairs = 0
+    for h, B in enumerate(sizes):
+        B = int(B)
+        pairs += B * (B + 1) // 2
+        if h >= 1:
+            pairs += B * (A + h * P)
+    pairs += T * N + T * (T + 1) // 2
+    return pairs
+
+
+def dense_pairs(cfg):
+    n = cfg.n_visual + cfg.n_text
+    return n * (n + 1) // 2
+
+
+def select_gather_bytes(cfg, sizes):
+    """Algorithmic HBM bytes of the score, select and gather kernels of one step."""
+    d, hq, hkv, H, P, R, N = cfg.head_dim, cfg.hq, cfg.hkv, cfg.n_hosts, cfg.passing, cfg.probe_r, cfg.n_visual
+    n_scored = int(sum(int(b) for b in sizes[:H - 1]))
+    score = n_scored * hkv * d * 2 + (H - 1) * R * hq * d * 2 + n_scored * hkv * 4
+    select = n_scored * hkv * 4 + (H - 1) * hkv * P * 4
+    gather = 2 * 2 * (H - 1) * hkv * P * d * 2 + (H - 1) * hkv * P * 4
+    return {"score": score, "select": select, "gather": gather}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle samples of this process's GPU during the timed region."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid.lower().replace("gpu-", "")
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9 or self.uuid not in parts[0].lower():
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle (baseline arm)
+class LazyF64:
+    """bf16 bit array viewed as float64, converted only where indexed (keeps the
+    oracle's memory to what it touches)."""
+
+    def __init__(self, bits):
+        self.bits = bits
+        self.shape = bits.shape
+
+    def __getitem__(self, key):
+        b = np.ascontiguousarray(self.bits[key], dtype=np.uint16)
+        return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def oracle_sample(cfg, g, seed, rows=512):
+    """One bounded oracle run: probe scoring + top-P selection of every host, then
+    the blockwise attention of one `rows`-row slice of a random host (all heads).
+    Returns (seconds for the whole workload, extrapolated by attended key pairs;
+    description; seconds actually spent)."""
+    from oracle import spava_oracle as orc
+    q, k, v = LazyF64(g["q"]), LazyF64(g["k"]), LazyF64(g["v"])
+    sizes = [int(x) for x in g["host_sizes"]]
+    off = orc.host_offsets(sizes)
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    t0 = time.perf_counter()
+    sel = None
+    if cfg.n_hosts > 1:
+        scores = orc.probe_scores(q, k, off, cfg.probe_r, scale)
+        sel = orc.select_passing(scores, off, cfg.anchor, cfg.passing)
+    t_sel = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    h = int(rng.integers(0, cfg.n_hosts))
+    a, e = int(off[h]), int(off[h + 1])
+    r0 = a + int(rng.integers(0, max(1, e - a - rows + 1)))
+    r1 = min(e, r0 + rows)
+    remote = (cfg.anchor + h * cfg.passing) if h >= 1 else 0
+    pairs_sample = sum(remote + (i - a + 1) for i in range(r0, r1))
+    t1 = time.perf_counter()
+    orc.approx_attention(q, k, v, off, cfg.anchor, sel, scale, row_range=(r0, r1))
+    t_att = time.perf_counter() - t1
+    total = t_sel + t_att * attended_pairs(cfg, sizes) / pairs_sample
+    desc = (f"fp64 numpy oracle: probe scoring + top-P selection of all hosts ({t_sel:.2f} s), then the "
+            f"blockwise attention of rows {r0}..{r1 - 1} (host {h}, all {cfg.hq} heads, {t_att:.2f} s), "
+            f"extrapolated to the whole layer by attended key pairs")
+    return total, desc, t_sel + t_att
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((int(x.get("num_threads", 1)) for x in info), default=os.cpu_count())
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, cfg):
+    g = generate(cfg)
+    NT = cfg.n_visual + cfg.n_text
+    for w in range(args.warmup):
+        oracle_sample(cfg, g, 100 + w, rows=args.ref_rows)
+    times = []
+    descs = []
+    wall = 0.0
+    for s in range(args.steps):
+        t, desc, w = oracle_sample(cfg, g, 1000 + s, rows=args.ref_rows)
+        times.append(t)
+        descs.append(desc)
+        wall += w
+    t_step = statistics.median(times)
+    value = NT / t_step
+    cores = blas_threads()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": workload_config(cfg),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": descs[-1] + f"; median of {args.steps} samples, {wall:.1f} s of CPU work"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfg):
+    return {"workload": cfg.name, "n_visual": cfg.n_visual, "n_text": cfg.n_text, "hosts": cfg.n_hosts,
+            "anchor": cfg.anchor, "passing": cfg.passing, "probe_r": cfg.probe_r, "hq": cfg.hq,
+            "hkv": cfg.hkv, "head_dim": cfg.head_dim, "kv": cfg.kv_kind, "seed": cfg.seed,
+            "l2": "inputs larger than L2 (no flush)", "parallelism": "replicas"}
+
+
+# ---------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="128k", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--dense", type=int, default=1, help="also time the dense causal kernel (0/1)")
+    ap.add_argument("--cpu-baseline", type=int, default=1)
+    ap.add_argument("--cpu-rows", type=int, default=1024)
+    ap.add_argument("--ref-rows", type=int, default=256)
+    args = ap.parse_args()
+    cfg = CONFIGS[args.config]
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, cfg)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import datetime
+
+    import sequence_approximate_attention_b200 as sab
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    g = generate(cfg)
+    sizes = [int(x) for x in g["host_sizes"]]
+    NT = cfg.n_visual + cfg.n_text
+    host = {x: torch.from_numpy(g[x].view(np.int16)).view(torch.bfloat16) for x in ("q", "k", "v")}
+    d_in = {x: host[x].to(dev) for x in host}
+    plan = sab.Plan(cfg.n_visual, cfg.n_text, cfg.n_hosts, sizes, cfg.anchor, cfg.passing, cfg.probe_r,
+                    cfg.hq, cfg.hkv, cfg.head_dim, device=dev)
+    ws = plan.new_workspace()
+    o = torch.empty_like(d_in["q"])
+    lse = torch.empty((cfg.hq, NT), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sab.attn_prefill(plan, d_in["q"], d_in["k"], d_in["v"], o=o, lse=lse, workspace=ws)
+        return sab.last_launch_count()
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    sab.check_device_error(plan, ws)
+
+    clocks = ClockSampler(str(torch.cuda.get_device_properties(dev).uuid))
+    plan.profile_begin(args.steps * 8 + 16)
+    launches = 0
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        launches += step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    ms_total = ev0.elapsed_time(ev1)
+    prof = plan.profile_read()
+    plan.profile_end()
+    sab.check_device_error(plan, ws)
+    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    value = world * NT * args.steps / (ms_total / 1e3)
+
+    # per-kernel averages over the timed steps
+    per = {}
+    for name, ms in prof:
+        per.setdefault(name, []).append(ms)
+    avg = {k: sum(v) / len(v) for k, v in per.items()}
+    peaks, peak_src = load_peaks()
+    pairs = attended_pairs(cfg, sizes)
+    flops = 4.0 * cfg.head_dim * cfg.hq * pairs
+    attn_ms = avg.get("attention", float("nan")) + avg.get("lse_merge", 0.0)
+    achieved = flops / (avg.get("attention", float("nan")) / 1e3) / 1e12
+    sgb = select_gather_bytes(cfg, sizes)
+    hbm = {}
+    for name in ("score", "select", "gather"):
+        if name in avg:
+            gbs = sgb[name] / (avg[name] / 1e3) / 1e9
+            hbm[name] = {"ms": avg[name], "bytes": sgb[name], "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]}
+    ssg_ms = sum(avg.get(n, 0.0) for n in ("score", "select", "gather"))
+    ssg_bytes = sum(sgb.values())
+    roofline = {
+        "bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved, "peak": peaks["bf16_tflops"],
+        "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+        "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)",
+        "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+        "frac_of_datasheet_2250": achieved / 2250.0,
+        "flops_per_launch": flops, "attended_pairs_per_head": pairs,
+        "launch_ms": avg.get("attention"),
+        "score_select_gather": {"ms": ssg_ms, "bytes": ssg_bytes,
+                                "GB/s": ssg_bytes / (ssg_ms / 1e3) / 1e9 if ssg_ms > 0 else None,
+                                "frac_of_hbm": (ssg_bytes / (ssg_ms / 1e3) / 1e9) / peaks["hbm_gbs"] if ssg_ms > 0 else None,
+                                "per_kernel": hbm},
+        "kernel_ms": avg,
+    }
+    step_tflops = flops / (ms_step / 1e3) / 1e12
+
+    # dense causal comparison on the same inputs
+    dense = None
+    if args.dense:
+        for _ in range(2):
+            sab.dense_causal(plan, d_in["q"], d_in["k"], d_in["v"], o=o, lse=lse, workspace=ws)
+        torch.cuda.synchronize(dev)
+        reps = 3
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            sab.dense_causal(plan, d_in["q"], d_in["k"], d_in["v"], o=o, lse=lse, workspace=ws)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        sab.check_device_error(plan, ws)
+        dms = e0.elapsed_time(e1) / reps
+        dfl = 4.0 * cfg.head_dim * cfg.hq * dense_pairs(cfg)
+        dense = {"ms": dms, "tokens/s": NT / (dms / 1e3), "TFLOP/s": dfl / (dms / 1e3) / 1e12,
+                 "frac": dfl / (dms / 1e3) / 1e12 / peaks["bf16_tflops"], "speedup_of_approx": dms / ms_step}
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = {x: host[x].pin_memory() for x in host}
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        l_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+        def e2e_step():
+            for x in ("q", "k", "v"):
+                d_in[x].copy_(pin[x], non_blocking=True)
+            sab.attn_prefill(plan, d_in["q"], d_in["k"], d_in["v"], o=o, lse=lse, workspace=ws)
+            o_h.copy_(o, non_blocking=True)
+            l_h.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * NT * args.e2e_steps / (float(te.item()) / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": sum(pin[x].numel() * 2 for x in pin),
+               "d2h_bytes_per_step": o_h.numel() * 2 + l_h.numel() * 4, "steps": args.e2e_steps}
+
+    cpu = None
+    if args.cpu_baseline and rank == 0 and world == 1:
+        t_full, desc, work = oracle_sample(cfg, g, 7, rows=args.cpu_rows)
+        cpu = {"value": NT / t_full, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc + f"; {work:.1f} s of CPU work", "host_cpus": os.cpu_count()}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "b200",
+            "config": workload_config(cfg),
+            "tflops_step": step_tflops, "tflops_step_frac": step_tflops / peaks["bf16_tflops"],
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clk, "dense_causal": dense,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    plan.close()
+
+
+if __name__ == "__main__":
+    main()

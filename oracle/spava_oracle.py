@@ -153,30 +153,34 @@ def _masked_softmax_attend(logits: np.ndarray, visible: np.ndarray, vals: np.nda
 
 def approx_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, off: np.ndarray,
                      anchor: int, sel: Optional[np.ndarray], scale: float,
-                     row_chunk: int = 512):
+                     row_chunk: int = 512, row_range=None):
     """Approximate attention of every row (host blocks + trailing text rows).
 
     Host h >= 1 attends to [anchor | passing of hosts < h | own block, causal];
     host 0 and text rows attend densely and causally.  Returns O float64
-    [tokens, hq, d] and lse float64 [hq, tokens] (natural log).
+    [tokens, hq, d] and lse float64 [hq, tokens] (natural log).  With
+    ``row_range=(r0, r1)`` only rows r0..r1-1 are computed (the rest stay NaN).
     """
     NT, hq, d = q.shape
     hkv = k.shape[1]
     G = _groups(hq, hkv)
     H = len(off) - 1
     N = int(off[-1])
-    O = np.empty((NT, hq, d), dtype=np.float64)
-    lse = np.empty((hq, NT), dtype=np.float64)
+    lo_row, hi_row = (0, NT) if row_range is None else (int(row_range[0]), int(row_range[1]))
+    O = np.full((NT, hq, d), np.nan, dtype=np.float64)
+    lse = np.full((hq, NT), np.nan, dtype=np.float64)
     for h in range(H):
         a, e = int(off[h]), int(off[h + 1])
+        if e <= lo_row or a >= hi_row:
+            continue
         for g in range(hkv):
             if h == 0:
                 remote = np.zeros(0, dtype=np.int64)
             else:
                 remote = np.concatenate([np.arange(0, anchor)] +
                                         [np.asarray(sel[hp, g], dtype=np.int64) for hp in range(h)])
-            for r0 in range(a, e, row_chunk):
-                r1 = min(e, r0 + row_chunk)
+            for r0 in range(max(a, lo_row), min(e, hi_row), row_chunk):
+                r1 = min(e, hi_row, r0 + row_chunk)
                 keys = np.concatenate([remote, np.arange(a, r1)])
                 visible = np.ones((r1 - r0, keys.size), dtype=bool)
                 visible[:, remote.size:] = np.arange(a, r1)[None, :] <= np.arange(r0, r1)[:, None]
@@ -184,8 +188,8 @@ def approx_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, off: np.ndarra
                 for c in range(g * G, (g + 1) * G):
                     logits = np.matmul(q[r0:r1, c, :], kk.T) * scale
                     O[r0:r1, c], lse[c, r0:r1] = _masked_softmax_attend(logits, visible, vv)
-    for r0 in range(N, NT, row_chunk):
-        r1 = min(NT, r0 + row_chunk)
+    for r0 in range(max(N, lo_row), min(NT, hi_row), row_chunk):
+        r1 = min(NT, hi_row, r0 + row_chunk)
         keys = np.arange(0, r1)
         visible = keys[None, :] <= np.arange(r0, r1)[:, None]
         for g in range(hkv):

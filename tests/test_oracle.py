@@ -191,6 +191,20 @@ def test_rows_formulation_matches_blockwise():
     np.testing.assert_allclose(L, full["lse"][heads, rows], rtol=1e-12, atol=1e-12)
 
 
+def test_row_range_matches_full():
+    cfg = CONFIGS["tiny"].with_(n_text=20, n_hosts=4)
+    g = generate(cfg)
+    q, k, v = (orc.bf16_bits_to_f64(g[x]) for x in ("q", "k", "v"))
+    scale = 1 / math.sqrt(cfg.head_dim)
+    full = orc.prefill(q, k, v, g["host_sizes"], cfg.anchor, cfg.passing, cfg.probe_r, scale=scale)
+    for r0, r1 in [(100, 300), (500, 532), (0, 7)]:
+        O, L = orc.approx_attention(q, k, v, full["offsets"], cfg.anchor, full["sel"], scale,
+                                    row_chunk=64, row_range=(r0, r1))
+        np.testing.assert_allclose(O[r0:r1], full["O"][r0:r1], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(L[:, r0:r1], full["lse"][:, r0:r1], rtol=1e-12, atol=1e-12)
+        assert np.isnan(O[r1:]).all() and np.isnan(O[:r0]).all()
+
+
 # ---------------------------------------------------------------- brute force: scores, select
 def test_scores_brute_force():
     rng = np.random.default_rng(3)
