@@ -151,6 +151,37 @@ spava_status spava_attn_prefill(const spava_plan* plan, const void* q, const voi
                                 int32_t* idx_out, void* ws, void* stream);
 
 /*
+ * spava_attn_prefill without a workspace, for callers that cannot allocate device
+ * memory at call time: frameworks whose device memory belongs to their own pooling
+ * allocator and that forbid a library to call cudaMalloc (an allocation outside the
+ * pool breaks its accounting, or fails outright under a hard memory cap), loops that
+ * cannot absorb the device-wide synchronisation cudaMalloc/cudaFree may cause, and
+ * interfaces that have no way to hand a scratch buffer to the library.  The paper
+ * has no counterpart of this entry point; it only changes where the scratch lives.
+ *
+ * The scratch is one static device array of SPAVA_NOALLOC_SCRATCH_BYTES (32 MiB)
+ * inside this library: every GPU on which the library's kernels are loaded holds it
+ * until the process exits.  This call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine); the inputs and outputs are the caller's, with the
+ * layouts of spava_attn_prefill.  The plan must have been created beforehand
+ * (spava_plan_create allocates its table once, at set-up).
+ *   First call on a device: it looks up the array's device address on the current
+ *   device (cudaGetSymbolAddress) and caches it; make that first call before any
+ *   stream capture.
+ *   Sizes: returns SPAVA_ERR_UNSUPPORTED, before enqueueing anything, when
+ *   spava_workspace_bytes(plan) exceeds SPAVA_NOALLOC_SCRATCH_BYTES.
+ *   Sharing: every call on a device uses the same array, which keeps the previous
+ *   call's contents (the call clears the part that must start at zero itself).  Calls
+ *   that overlap on the GPU (other streams, threads or plans) race on it: serialise
+ *   them.  The scores, selection and error word stay in the array; a bounded-wait
+ *   timeout inside this call is therefore not reported (use spava_attn_prefill with a
+ *   workspace and spava_check_device_error when that check is needed).
+ */
+#define SPAVA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+spava_status spava_attn_prefill_noalloc(const spava_plan* plan, const void* q, const void* k,
+                                        const void* v, void* o, float* lse, void* stream);
+
+/*
  * Dense causal attention over all N+T tokens on the same kernel (the standard
  * FlashAttention the method degenerates to on one host; the comparison kernel).
  * Layouts as above.

@@ -30,6 +30,8 @@ SIGNATURES = {
                                        c_void_p, c_void_p]),
     "spava_attn_prefill": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                      c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "spava_attn_prefill_noalloc": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                             c_void_p, c_void_p]),
     "spava_dense_causal": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                      c_void_p, c_void_p, c_void_p]),
     "spava_check_device_error": (c_int32, [c_void_p, c_void_p, c_void_p]),

@@ -599,6 +599,56 @@ spava_status spava_attn_prefill(const spava_plan* p, const void* q, const void* 
   return ok();
 }
 
+}  // extern "C"
+
+// Scratch of spava_attn_prefill_noalloc: one array per device holding the
+// library's kernels, shared by every call on that device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SPAVA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on device `dev` (which must be current): in
+// host code the symbol is only a host-side stand-in, so the address is looked up
+// once per device and cached.
+spava_status noalloc_scratch_address(int dev, void** out) {
+  if (dev < 0 || dev >= kMaxDevices) return fail(SPAVA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void* addr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
+    if (e != cudaSuccess || !addr)
+      return fail(SPAVA_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
+    g_noalloc_addr[dev] = addr;
+  }
+  *out = g_noalloc_addr[dev];
+  return SPAVA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+spava_status spava_attn_prefill_noalloc(const spava_plan* p, const void* q, const void* k, const void* v, void* o,
+                                        float* lse, void* stream) {
+  if (!p) return fail(SPAVA_ERR_INVALID_ARG, "plan is NULL");
+  if (p->ws_total > SPAVA_NOALLOC_SCRATCH_BYTES)
+    return fail(SPAVA_ERR_UNSUPPORTED,
+                "this plan needs %zu bytes of scratch, the static scratch holds %u; "
+                "use spava_attn_prefill with a workspace",
+                p->ws_total, SPAVA_NOALLOC_SCRATCH_BYTES);
+  int dev = -1;
+  SPAVA_CUDA(cudaGetDevice(&dev));
+  if (dev != p->device) return fail(SPAVA_ERR_INVALID_ARG, "current device %d differs from the plan's device %d", dev, p->device);
+  void* ws = nullptr;
+  spava_status s = noalloc_scratch_address(dev, &ws);
+  if (s != SPAVA_OK) return s;
+  return spava_attn_prefill(p, q, k, v, o, lse, nullptr, nullptr, ws, stream);
+}
+
 spava_status spava_dense_causal(const spava_plan* p, const void* q, const void* k, const void* v, void* o, float* lse,
                                 void* ws, void* stream) {
   spava_status s;
