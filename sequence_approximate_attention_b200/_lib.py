@@ -61,12 +61,13 @@ def _status_name(s: int) -> str:
 
 
 def load(build_if_missing: bool = True):
-    """Load libspava.so (building it first if it is missing or older than its sources)."""
+    """Load libspava.so (building it first if it is missing or older than its sources).
+    SPAVA_LIB_PATH, if set, names another build of the same library to load instead."""
     global _LIB
     if _LIB is not None:
         return _LIB
-    path = _build.LIB_PATH
-    if build_if_missing and _build.is_stale():
+    path = os.environ.get("SPAVA_LIB_PATH") or _build.LIB_PATH
+    if path == _build.LIB_PATH and build_if_missing and _build.is_stale():
         _build.build()
     if not os.path.exists(path):
         raise ImportError(f"libspava.so is not built ({path}); run "

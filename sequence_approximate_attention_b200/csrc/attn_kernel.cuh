@@ -68,6 +68,13 @@ struct AttnParams {
   int stall_producer;
 };
 
+// Pairs (out of every 8) whose exp2 runs on the FMA/ALU pipes (exp2_poly2) instead
+// of MUFU.  Measured on B200 at this tile shape (two 128-row tiles, 128-key KV
+// tiles, one softmax warp per 32 rows), every share above 0 was slower: each
+// warp's softmax is bound by its own issue and latency chain, not by MUFU
+// throughput, so the extra instructions cost more than the MUFU time they free.
+constexpr int kPolyPairsOf8 = 0;
+
 template <int D>
 struct AttnShape {
   static_assert(D == 64 || D == 128, "head_dim");
@@ -83,6 +90,7 @@ struct AttnShape {
   static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);
   static constexpr uint32_t kIdescO = idesc_bf16_f32(128, D, 0, 1);
   static constexpr int kThreads = 384;
+
   __device__ static constexpr uint32_t tmem_s(int i) { return static_cast<uint32_t>(i * 128); }
   __device__ static constexpr uint32_t tmem_o(int i) { return static_cast<uint32_t>(256 + i * D); }
 };
@@ -138,7 +146,7 @@ __device__ __forceinline__ AttnItem load_item(const AttnItem* items, int idx) {
 
 // Wait on a barrier that no timeout or abort may cut short (draining copies in
 // flight before the CTA exits); still bounded.
-__device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
   const uint64_t t0 = global_timer_ns();
   for (;;) {
     if (mbar_test(bar, parity)) return true;
@@ -182,7 +190,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, 128);
+      mbar_init(p_full + i, 4);  // one arrival per softmax warp
       mbar_init(o_full + i, 1);
     }
     mbar_init(drain, 1);
@@ -201,7 +209,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, p.err_word, p.wait_limit_ns};
   const int G = gridDim.x, cta = blockIdx.x;
-
+  if (warp < 4) {
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     int ring = 0, m = 0, q_issued = 0;
@@ -271,22 +279,30 @@ __global__ void __launch_bounds__(384, 1)
     int ring = 0, m = 0;
     uint32_t pc0 = 0, pc1 = 0;
     bool ok = true, issued_any = false;
+    // Descriptor bases built once; per MMA only the start-address field moves (it is
+    // the low 14 bits of the descriptor, in 16-byte units, and never carries:
+    // shared memory addresses stay below 256 KB).  Keeping the issue path down to
+    // a handful of integer adds per MMA matters: this one thread feeds the tensor
+    // core 32 MMAs per KV tile.
+    const uint64_t q_desc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t kv_desc0 = sdesc_sw128(smem_u32(sKV), 16, 1024);
+    const uint64_t v_desc0 = sdesc_sw128(smem_u32(sKV), S::kHalfBytes, 1024);
+    constexpr uint32_t kTileStep = S::kTileBytes >> 4;
     auto issue_s = [&](int i, int slot) {
-      const uint32_t qa = smem_u32(sQ + i * S::kTileBytes);
-      const uint32_t ka = smem_u32(sKV + slot * S::kTileBytes);
+      const uint64_t qd = q_desc0 + static_cast<uint32_t>(i) * kTileStep;
+      const uint64_t kd = kv_desc0 + static_cast<uint32_t>(slot) * kTileStep;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * S::kHalfBytes + (kk & 3) * 32;
-        mma_ss(tmem + S::tmem_s(i), sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), S::kIdescS,
-               kk > 0 ? 1u : 0u);
+        const uint32_t off = ((kk >> 2) * S::kHalfBytes + (kk & 3) * 32) >> 4;
+        mma_ss(tmem + S::tmem_s(i), qd + off, kd + off, S::kIdescS, kk > 0 ? 1u : 0u);
       }
     };
     auto issue_pv = [&](int i, int slot, bool acc) {
-      const uint32_t va = smem_u32(sKV + slot * S::kTileBytes);
+      const uint64_t vd = v_desc0 + static_cast<uint32_t>(slot) * kTileStep;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        mma_ts(tmem + S::tmem_o(i), tmem + S::tmem_s(i) + kk * 8, sdesc_sw128(va + kk * 2048, S::kHalfBytes, 1024),
-               S::kIdescO, (acc || kk > 0) ? 1u : 0u);
+        mma_ts(tmem + S::tmem_o(i), tmem + S::tmem_s(i) + kk * 8, vd + ((kk * 2048) >> 4), S::kIdescO,
+               (acc || kk > 0) ? 1u : 0u);
       }
     };
     for (int r = 0; ok; ++r) {
@@ -378,7 +394,8 @@ __global__ void __launch_bounds__(384, 1)
       }
       __syncwarp();
     }
-  } else if (warp >= 4) {
+  }
+  } else {
     // ------------------------------------------------------------ softmax / epilogue
     const int i = (warp - 4) >> 2;  // Q tile of this warpgroup
     const int qd = warp & 3;        // TMEM lane quarter
@@ -408,20 +425,22 @@ __global__ void __launch_bounds__(384, 1)
         const bool causal = (sg.flags & kSegCausal) != 0;
         uint32_t sr[128];
         tmem_ld_x128(tl + S::tmem_s(i), sr);
-        float tmax = -INFINITY;
         if (valid < 128 || (causal && kpos0 + 127 > qrow0)) {
           int lim = valid;
           if (causal) lim = min(lim, qpos - kpos0 + 1);
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            float x = c < lim ? __uint_as_float(sr[c]) : -INFINITY;
-            sr[c] = __float_as_uint(x);
-            tmax = fmaxf(tmax, x);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) tmax = fmaxf(tmax, __uint_as_float(sr[c]));
+          for (int c = 0; c < 128; ++c)
+            if (c >= lim) sr[c] = 0xff800000u;  // -inf
         }
+        // Row max: eight independent chains of three-input maxes, then a tree.
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[k + 8]));
+#pragma unroll
+        for (int c = 16; c < 128; c += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
+        const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
         const float m_tile = tmax * sl2;
         float alpha = 1.0f;
         bool rescale = false;
@@ -436,17 +455,20 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
-        float rs = 0.f;
-        // P = exp2(s * scale_log2 - m) packed to bf16 pairs in place: pair c lands in
-        // sr[c] after sr[2c], sr[2c+1] have been read.
+        // P = exp2(s * scale_log2 - m) on the MUFU unit, packed to bf16 pairs in place
+        // (pair c lands in sr[c] after sr[2c], sr[2c+1] have been read); the scale-
+        // subtract and the row sum run as packed fp32 pairs in four chains.
+        const float2 sl2x2 = make_float2(sl2, sl2), negm = make_float2(-m_use, -m_use);
+        float2 rs[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * c]), sl2, -m_use));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m_use));
-          rs += p0 + p1;
-          sr[c] = pack_bf16x2(p0, p1);
+          const float2 x = ffma2(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2x2, negm);
+          const float2 pp = ((c & 7) < kPolyPairsOf8) ? exp2_poly2(x) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+          rs[c & 3] = fadd2(rs[c & 3], pp);
+          sr[c] = pack_bf16x2(pp.x, pp.y);
         }
-        l_run = l_run * alpha + rs;
+        const float2 r01 = fadd2(rs[0], rs[1]), r23 = fadd2(rs[2], rs[3]), r = fadd2(r01, r23);
+        l_run = l_run * alpha + (r.x + r.y);
         tmem_st_x64(tl + S::tmem_s(i), *reinterpret_cast<uint32_t(*)[64]>(sr));
         if (rescale) {
           // O_i holds the sum up to tile j-1 (its MMA finished before S_i(j) did).
@@ -460,7 +482,8 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         tc_fence_before();
-        mbar_arrive(p_full + i);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + i);
       }
       if (!ok) break;
       ok = __all_sync(FULL, mbar_wait(o_full + i, oc & 1, wc, kErrWaitMma));

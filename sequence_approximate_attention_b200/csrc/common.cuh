@@ -73,8 +73,7 @@ struct WaitCtx {
 // Wait for the phase of `bar` with parity `parity` to complete.  Returns false
 // (without completing) if the CTA is aborting or the limit ran out; in the second
 // case this thread raises the abort flag and records `code`.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w, uint32_t code) {
-  if (mbar_test(bar, parity)) return true;
+__device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const WaitCtx& w, uint32_t code) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t spin = 1;; ++spin) {
     if (mbar_test(bar, parity)) return true;
@@ -88,6 +87,11 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Wai
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w, uint32_t code) {
+  if (mbar_test(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, w, code);
 }
 
 // ---------------------------------------------------------------- TMA
@@ -177,11 +181,87 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Per-warpgroup register budget (all four warps of a warpgroup execute the same
+// call).  The budgets of all warpgroups must add up to at most the registers the
+// CTA was launched with, or the increase waits forever.
+template <uint32_t kRegs>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
 // ---------------------------------------------------------------- math helpers
 __device__ __forceinline__ float fast_exp2(float x) {  // MUFU ex2 (ftz); exp2(-inf) = +0
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+#include "exp2_poly.inc"
+
+// 2^x on the FMA/ALU pipes, for the part of the softmax that is kept off the MUFU
+// unit: Cody-Waite style range reduction 2^x = 2^round(x) * 2^f, f in [-1/2, 1/2],
+// with round(x) taken from the low mantissa bits of x + 1.5*2^23, and a degree-3
+// minimax polynomial for 2^f (coefficients from gen_exp2_poly.py, max relative
+// error 7.5e-5).  Inputs below -126 are clamped (the result is then ~1e-38 instead
+// of 0, which no softmax sum can notice).
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = __fadd_rn(x, 12582912.0f);
+  const float r = __fsub_rn(t, 12582912.0f);
+  const float f = __fsub_rn(x, r);
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Packed fp32 pair arithmetic (sm_100 f32x2 forms) and a three-input max: they
+// halve the instruction count of the softmax's scale-subtract, row sum and row max.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// exp2_poly on a pair, in packed fp32 arithmetic: two clamps, two packed adds for the
+// range reduction, one packed fma for the fraction, three packed fmas for the
+// polynomial and a shift-add per element to apply 2^round(x).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 big = make_float2(12582912.0f, 12582912.0f);
+  const float2 t = fadd2(x, big);
+  const float2 r = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = ffma2(r, make_float2(-1.0f, -1.0f), x);
+  float2 p = ffma2(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  p = ffma2(p, f, make_float2(kExp2C1, kExp2C1));
+  p = ffma2(p, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

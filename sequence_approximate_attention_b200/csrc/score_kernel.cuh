@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(q_full + b, 1);
       mbar_init(q_empty + b, 1);
       mbar_init(acc_full + b, 1);
-      mbar_init(acc_empty + b, 128);
+      mbar_init(acc_empty + b, 4);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -236,7 +236,8 @@ __global__ void __launch_bounds__(256, 1)
           }
         }
         tc_fence_before();
-        mbar_arrive(acc_empty + b);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty + b);
       }
       if (!ok) break;
       if (j < e) p.scores[static_cast<size_t>(it.y) * p.n_visual + j] = mx * p.scale;
