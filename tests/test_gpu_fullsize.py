@@ -1,0 +1,157 @@
+"""Parity at the full sizes of the five workloads, through the C ABI, in the launch
+configuration bench.py times (one plan, one workspace, one spava_attn_prefill).
+
+Every score of hosts 0..H-2 is checked against the fp64 oracle; the selection is
+checked bit-exactly against the oracle's selection on the GPU's own fp32 scores and
+for near-tie-only differences against the fp64 selection; O and lse are checked on
+sampled (row, head) outputs -- block starts, tile boundaries, probe rows, block
+ends, text rows and random rows -- against the oracle re-run with the GPU's
+indices.  The 256k workload also runs the dense causal kernel on the same inputs.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import spava_oracle as orc
+from workloads import CONFIGS, generate
+
+from .helpers import LSE_TOL, O_TOL, check_selection_vs_fp64, to_device_bf16
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+sab = pytest.importorskip("sequence_approximate_attention_b200")
+
+
+class LazyF64:
+    """bf16 bits viewed as float64, converted where indexed (keeps host memory low)."""
+
+    def __init__(self, bits):
+        self.bits = bits
+        self.shape = bits.shape
+
+    def __getitem__(self, key):
+        b = np.ascontiguousarray(self.bits[key], dtype=np.uint16)
+        return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def _score_tolerance_and_ref(q, k, off, R, scale, hosts):
+    hq, hkv = q.shape[1], k.shape[1]
+    G = hq // hkv
+    ref = {}
+    tol = {}
+    for h in hosts:
+        a, e = int(off[h]), int(off[h + 1])
+        keys = np.arange(a, e)
+        rows = np.arange(e - R, e)
+        vis = rows[:, None] >= keys[None, :]
+        qh = q[e - R:e]                                   # [R, hq, d]
+        for g in range(hkv):
+            qg = qh[:, g * G:(g + 1) * G, :].reshape(-1, qh.shape[2])   # [(R*G), d], row = (r, c)
+            kb = k[a:e, g, :]
+            s = (qg @ kb.T).reshape(R, G, -1) * scale
+            s = np.where(vis[:, None, :], s, -np.inf)
+            ref[(h, g)] = s.max(axis=(0, 1))
+            tol[(h, g)] = 1e-5 * scale * (np.abs(qg) @ np.abs(kb).T).max(axis=0) + 1e-6
+    return ref, tol
+
+
+def _sample_rows(cfg, off, rng, n_random=48):
+    rows = set()
+    for h in range(cfg.n_hosts):
+        a, e = int(off[h]), int(off[h + 1])
+        for r in (a, a + 1, a + 127, a + 128, a + 255, a + 256, e - cfg.probe_r, e - 2, e - 1):
+            if a <= r < e:
+                rows.add(r)
+    for r in (cfg.n_visual, cfg.n_visual + cfg.n_text // 2, cfg.n_visual + cfg.n_text - 1):
+        if cfg.n_text and r < cfg.n_visual + cfg.n_text:
+            rows.add(r)
+    rows.update(int(x) for x in rng.integers(0, cfg.n_visual + cfg.n_text, n_random))
+    rows = sorted(rows)
+    heads = [int((i * 7 + 3) % cfg.hq) for i in range(len(rows))]
+    return rows, heads
+
+
+@pytest.fixture(scope="module", params=["qwen64k", "128k", "stress", "256k"])
+def fullsize_run(request):
+    cfg = CONFIGS[request.param]
+    g = generate(cfg)
+    sizes = [int(x) for x in g["host_sizes"]]
+    dev = {x: to_device_bf16(g[x]) for x in ("q", "k", "v")}
+    plan = sab.Plan(cfg.n_visual, cfg.n_text, cfg.n_hosts, sizes, cfg.anchor, cfg.passing, cfg.probe_r,
+                    cfg.hq, cfg.hkv, cfg.head_dim)
+    ws = plan.new_workspace()
+    scores = torch.empty((cfg.hkv, cfg.n_visual), dtype=torch.float32, device="cuda")
+    idx = torch.empty(plan.idx_shape(), dtype=torch.int32, device="cuda")
+    o, lse = sab.attn_prefill(plan, dev["q"], dev["k"], dev["v"], scores_out=scores, idx_out=idx, workspace=ws)
+    sab.check_device_error(plan, ws)
+    res = {"cfg": cfg, "g": g, "sizes": sizes, "plan": plan, "dev": dev, "ws": ws,
+           "scores": scores.cpu().numpy(), "idx": idx.cpu().numpy().astype(np.int64),
+           "o": o, "lse": lse}
+    yield res
+    plan.close()
+    del dev, o, lse
+    torch.cuda.empty_cache()
+
+
+def test_fullsize_scores_and_selection(fullsize_run):
+    r = fullsize_run
+    cfg = r["cfg"]
+    off = orc.host_offsets(r["sizes"])
+    q, k = LazyF64(r["g"]["q"]), LazyF64(r["g"]["k"])
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    hosts = range(cfg.n_hosts - 1)
+    ref, tol = _score_tolerance_and_ref(q, k, off, cfg.probe_r, scale, hosts)
+    sc = r["scores"]
+    ref64 = np.full_like(sc, np.nan, dtype=np.float64)
+    for (h, g), v in ref.items():
+        a, e = int(off[h]), int(off[h + 1])
+        err = np.abs(sc[g, a:e] - v)
+        assert (err <= tol[(h, g)]).all(), (cfg.name, h, g, float(err.max()))
+        ref64[g, a:e] = v
+    np.testing.assert_array_equal(r["idx"], orc.select_passing(sc, off, cfg.anchor, cfg.passing))
+    # fp64 selection: differences only at near-ties (rows of host H-1 are unused)
+    ref64[:, int(off[cfg.n_hosts - 1]):] = 0.0
+    check_selection_vs_fp64(r["idx"], ref64, off, cfg.anchor, cfg.passing)
+
+
+def test_fullsize_sampled_outputs(fullsize_run):
+    r = fullsize_run
+    cfg = r["cfg"]
+    off = orc.host_offsets(r["sizes"])
+    q, k, v = (LazyF64(r["g"][x]) for x in ("q", "k", "v"))
+    rng = np.random.default_rng(cfg.seed)
+    rows, heads = _sample_rows(cfg, off, rng)
+    O_ref, L_ref = orc.attention_rows(q, k, v, off, cfg.anchor, r["idx"], 1.0 / math.sqrt(cfg.head_dim), rows, heads)
+    rt = torch.tensor(rows, device="cuda")
+    ht = torch.tensor(heads, device="cuda")
+    o = r["o"][rt, ht].float().cpu().numpy()
+    lse = r["lse"][ht, rt].cpu().numpy()
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    do = np.abs(o - O_ref).max()
+    dl = np.abs(lse - L_ref).max()
+    assert do <= O_TOL and dl <= LSE_TOL, (cfg.name, do, dl)
+    # every output is finite (no NaN/inf anywhere in the full tensors)
+    assert torch.isfinite(r["o"].float()).all().item() and torch.isfinite(r["lse"]).all().item()
+
+
+def test_fullsize_dense_causal_256k(fullsize_run):
+    r = fullsize_run
+    cfg = r["cfg"]
+    if cfg.name != "256k":
+        pytest.skip("the dense causal comparison runs on the 256k workload")
+    dev = r["dev"]
+    o, lse = sab.dense_causal(r["plan"], dev["q"], dev["k"], dev["v"], workspace=r["ws"])
+    sab.check_device_error(r["plan"], r["ws"])
+    off = orc.host_offsets([cfg.n_visual])   # one host: dense causal
+    q, k, v = (LazyF64(r["g"][x]) for x in ("q", "k", "v"))
+    NT = cfg.n_visual + cfg.n_text
+    rows = [0, 1, 127, 128, 4095, 100000, 200000, NT - 300, NT - 1]
+    heads = [(i * 5) % cfg.hq for i in range(len(rows))]
+    O_ref, L_ref = orc.attention_rows(q, k, v, off, 0, None, 1.0 / math.sqrt(cfg.head_dim), rows, heads)
+    rt, ht = torch.tensor(rows, device="cuda"), torch.tensor(heads, device="cuda")
+    do = np.abs(o[rt, ht].float().cpu().numpy() - O_ref).max()
+    dl = np.abs(lse[ht, rt].cpu().numpy() - L_ref).max()
+    assert do <= O_TOL and dl <= LSE_TOL, (do, dl)
