@@ -63,7 +63,7 @@ def select_gather_bytes(cfg, sizes):
     score = n_scored * hkv * d * 2 + (H - 1) * R * hq * d * 2 + n_scored * hkv * 4
     select = n_scored * hkv * 4 + (H - 1) * hkv * P * 4
     gather = 2 * 2 * (H - 1) * hkv * P * d * 2 + (H - 1) * hkv * P * 4
-    return {"score": score, "select": select, "gather": gather}
+    return {"score": score, "select": select, "gather": gather, "select_gather": select + gather}
 
 
 def load_peaks():
@@ -324,12 +324,13 @@ def main():
     achieved = flops / (avg.get("attention", float("nan")) / 1e3) / 1e12
     sgb = select_gather_bytes(cfg, sizes)
     hbm = {}
-    for name in ("score", "select", "gather"):
+    for name in ("score", "select", "gather", "select_gather"):
         if name in avg:
             gbs = sgb[name] / (avg[name] / 1e3) / 1e9
             hbm[name] = {"ms": avg[name], "bytes": sgb[name], "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]}
-    ssg_ms = sum(avg.get(n, 0.0) for n in ("score", "select", "gather"))
-    ssg_bytes = sum(sgb.values())
+    ssg_names = [n for n in ("score", "select", "gather", "select_gather") if n in avg]
+    ssg_ms = sum(avg[n] for n in ssg_names)
+    ssg_bytes = sum(sgb[n] for n in ssg_names)
     roofline = {
         "bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved, "peak": peaks["bf16_tflops"],
         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,

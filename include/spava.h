@@ -213,7 +213,7 @@ int32_t spava_profile_read(spava_plan* plan, int32_t* labels, float* ms, int32_t
 spava_status spava_profile_end(spava_plan* plan);
 
 /* Name of a kernel label: 0 score, 1 select, 2 gather, 3 attention (prefill),
- * 4 lse merge, 5 attention (dense causal). */
+ * 4 lse merge, 5 attention (dense causal), 6 select + gather (fused, prefill). */
 const char* spava_kernel_name(int32_t label);
 
 /* Static text of a status code. */

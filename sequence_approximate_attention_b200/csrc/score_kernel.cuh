@@ -33,29 +33,55 @@ struct ScoreParams {
   float* scores;     // [hkv][N]
   unsigned int* err_word;
   uint64_t wait_limit_ns;
+  // shared-memory pipeline, sized on the host: probe-query buffers (1 when every
+  // (host, group) fits one chunk, else 2) and K-tile stages filling the rest
+  int q_bufs;
+  int q_buf_bytes;
+  int k_stages;
 };
 
 template <int D>
 struct ScoreShape {
   static constexpr int kHalves = D / 64;
   static constexpr int kKTileBytes = kHalves * 128 * 128;  // 128 keys
-  static constexpr int kQBufBytes = kHalves * 256 * 128;   // up to 256 probe rows
-  static constexpr int kKOff = 0;
-  static constexpr int kQOff = 2 * kKTileBytes;
-  static constexpr int kBarOff = kQOff + 2 * kQBufBytes;
-  static constexpr int kSmemBytes = kBarOff + 256 + 1024;
+  static constexpr int kMaxStages = 8;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kMaxLocalItems = 512;  // item metadata cached in shared memory
+  static constexpr int kItemBytes = kMaxLocalItems * 16;
+  static constexpr int kSmemMax = 232448;  // opt-in limit per CTA on sm_100
   static constexpr uint32_t kTmemCols = 512;
+  // Bytes of dynamic shared memory for a given pipeline (plus alignment slack).
+  static constexpr int smem_bytes(int q_bufs, int q_buf_bytes, int k_stages) {
+    return q_bufs * q_buf_bytes + k_stages * kKTileBytes + kBarBytes + kItemBytes + 1024;
+  }
 };
 
-// Chunk-use u of this CTA needs a fresh load of probe queries iff the buffer it
-// maps to (u & 1) last held a different (host, group, chunk).
-__device__ __forceinline__ bool score_needs_load(const ScoreParams& p, int first, int u) {
-  if (u < 2) return true;
-  const int a = u, b = u - 2;
-  const int ia = first + a / p.n_chunks, ib = first + b / p.n_chunks;
-  if (a % p.n_chunks != b % p.n_chunks) return true;
-  const int4 x = __ldg(p.items + ia), y = __ldg(p.items + ib);
+// Chunk-use (li, c) of this CTA -- item li, probe chunk c, use u = li*n_chunks + c --
+// needs a fresh load of probe queries iff the buffer it maps to (u % q_bufs) last
+// held a different (host, group, chunk).  `items` is the CTA's item range in shared
+// memory.  Written without integer division (q_bufs <= 2): this runs on the MMA
+// thread's critical path once per chunk.
+__device__ __forceinline__ bool score_needs_load(const ScoreParams& p, const int4* items, int li, int c) {
+  int cb = c - p.q_bufs, lb = li;
+  while (cb < 0) {
+    cb += p.n_chunks;
+    --lb;
+  }
+  if (lb < 0) return true;  // first uses of each buffer
+  if (cb != c) return true;   // the buffer held another chunk of the probe
+  const int4 x = items[li], y = items[lb];
   return x.x != y.x || x.y != y.y;
+}
+
+// The use that comes q_bufs uses after (li, c), as (item, chunk).
+__device__ __forceinline__ void score_next_use(const ScoreParams& p, int li, int c, int* ln, int* cn) {
+  int cc = c + p.q_bufs, l = li;
+  while (cc >= p.n_chunks) {
+    cc -= p.n_chunks;
+    ++l;
+  }
+  *ln = l;
+  *cn = cc;
 }
 
 template <int D>
@@ -66,24 +92,28 @@ __global__ void __launch_bounds__(256, 1)
   constexpr uint32_t FULL = 0xffffffffu;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sK = smem + S::kKOff;
-  uint8_t* sQ = smem + S::kQOff;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
-  uint64_t* k_full = bars + 0;      // [2]
-  uint64_t* k_empty = bars + 2;     // [2]
-  uint64_t* q_full = bars + 4;      // [2]
-  uint64_t* q_empty = bars + 6;     // [2]
-  uint64_t* acc_full = bars + 8;    // [2]
-  uint64_t* acc_empty = bars + 10;  // [2]
-  uint64_t* drain = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  const int n_stages = p.k_stages;
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + p.q_bufs * p.q_buf_bytes;   // q_buf_bytes is a multiple of 1024
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sK + n_stages * S::kKTileBytes);
+  uint64_t* k_full = bars + 0;                   // [kMaxStages]
+  uint64_t* k_empty = k_full + S::kMaxStages;    // [kMaxStages]
+  uint64_t* q_full = k_empty + S::kMaxStages;    // [2]
+  uint64_t* q_empty = q_full + 2;                // [2]
+  uint64_t* acc_full = q_empty + 2;              // [2]
+  uint64_t* acc_empty = acc_full + 2;            // [2]
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int4* s_items = reinterpret_cast<int4*>(reinterpret_cast<uint8_t*>(bars) + S::kBarBytes);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < n_stages; ++b) {
       mbar_init(k_full + b, 1);
       mbar_init(k_empty + b, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(q_full + b, 1);
       mbar_init(q_empty + b, 1);
       mbar_init(acc_full + b, 1);
@@ -106,16 +136,19 @@ __global__ void __launch_bounds__(256, 1)
   const int n_local = last - first;
   const int total_uses = n_local * p.n_chunks;
   const int G = p.group;
+  // The host sizes the grid so that every CTA's range fits the shared-memory cache.
+  for (int t = threadIdx.x; t < n_local; t += blockDim.x) s_items[t] = __ldg(p.items + first + t);
+  __syncthreads();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    int qloads[2] = {0, 0}, kloads[2] = {0, 0};
+    int qloads[2] = {0, 0};
+    int slot = 0, use = 0;  // K stage and how often it was filled before (no division)
     bool ok = true;
     for (int li = 0; li < n_local && ok; ++li) {
-      const int4 it = __ldg(p.items + first + li);
-      const int slot = li & 1;
-      if (li >= 2) {
-        ok = __all_sync(FULL, mbar_wait(k_empty + slot, ((li >> 1) - 1) & 1, wc, kErrWaitRelease));
+      const int4 it = s_items[li];
+      if (use > 0) {
+        ok = __all_sync(FULL, mbar_wait(k_empty + slot, (use - 1) & 1, wc, kErrWaitRelease));
         if (!ok) break;
       }
       if (lane == 0) {
@@ -124,10 +157,13 @@ __global__ void __launch_bounds__(256, 1)
           tma_load_3d(sK + slot * S::kKTileBytes + hh * 128 * 128, &tmK, k_full + slot, hh * 64, it.y, it.z);
       }
       __syncwarp();
-      ++kloads[slot];
+      if (++slot == n_stages) {
+        slot = 0;
+        ++use;
+      }
       for (int c = 0; c < p.n_chunks; ++c) {
-        const int u = li * p.n_chunks + c, b = u & 1;
-        if (!score_needs_load(p, first, u)) continue;
+        const int u = li * p.n_chunks + c, b = u & (p.q_bufs - 1);
+        if (!score_needs_load(p, s_items, li, c)) continue;
         if (qloads[b] > 0) {
           ok = __all_sync(FULL, mbar_wait(q_empty + b, (qloads[b] - 1) & 1, wc, kErrWaitRelease));
           if (!ok) break;
@@ -135,7 +171,7 @@ __global__ void __launch_bounds__(256, 1)
         if (lane == 0) {
           mbar_arrive_expect_tx(q_full + b, static_cast<uint32_t>(S::kHalves * p.chunk_tokens * G * 128));
           for (int hh = 0; hh < S::kHalves; ++hh)
-            tma_load_3d(sQ + b * S::kQBufBytes + hh * (p.chunk_tokens * G * 128), &tmQp, q_full + b, hh * 64,
+            tma_load_3d(sQ + b * p.q_buf_bytes + hh * (p.chunk_tokens * G * 128), &tmQp, q_full + b, hh * 64,
                         it.y * G, it.w - p.probe_r + c * p.chunk_tokens);
         }
         __syncwarp();
@@ -145,10 +181,12 @@ __global__ void __launch_bounds__(256, 1)
     if (!ok) {
       // Abort: let every copy this warp issued land before the CTA exits.
       if (lane == 0) {
-        for (int b = 0; b < 2; ++b) {
-          if (kloads[b] > 0) mbar_wait_drain(k_full + b, (kloads[b] - 1) & 1, wc);
-          if (qloads[b] > 0) mbar_wait_drain(q_full + b, (qloads[b] - 1) & 1, wc);
+        for (int b = 0; b < n_stages; ++b) {
+          const int uses = use + (b < slot ? 1 : 0);  // loads issued into stage b
+          if (uses > 0) mbar_wait_drain(k_full + b, (uses - 1) & 1, wc);
         }
+        for (int b = 0; b < 2; ++b)
+          if (qloads[b] > 0) mbar_wait_drain(q_full + b, (qloads[b] - 1) & 1, wc);
       }
       __syncwarp();
     }
@@ -156,19 +194,21 @@ __global__ void __launch_bounds__(256, 1)
     // ------------------------------------------------------------ MMA issuer
     int qloads[2] = {0, 0};
     bool ok = true, issued_any = false;
+    int slot = 0, kphase = 0;
     for (int li = 0; li < n_local && ok; ++li) {
-      const int slot = li & 1;
-      ok = __all_sync(FULL, mbar_wait(k_full + slot, (li >> 1) & 1, wc, kErrWaitLoad));
+      ok = __all_sync(FULL, mbar_wait(k_full + slot, kphase, wc, kErrWaitLoad));
       if (!ok) break;
       for (int c = 0; c < p.n_chunks; ++c) {
-        const int u = li * p.n_chunks + c, b = u & 1;
-        if (score_needs_load(p, first, u)) {
-          ok = __all_sync(FULL, mbar_wait(q_full + b, qloads[b] & 1, wc, kErrWaitLoad));
-          ++qloads[b];
+        const int u = li * p.n_chunks + c;
+        const int qb = u & (p.q_bufs - 1);  // probe-query buffer (q_bufs is 1 or 2)
+        const int ab = u & 1;               // TMEM accumulator
+        if (score_needs_load(p, s_items, li, c)) {
+          ok = __all_sync(FULL, mbar_wait(q_full + qb, qloads[qb] & 1, wc, kErrWaitLoad));
+          ++qloads[qb];
           if (!ok) break;
         }
         if (u >= 2) {
-          ok = __all_sync(FULL, mbar_wait(acc_empty + b, ((u >> 1) - 1) & 1, wc, kErrWaitMma));
+          ok = __all_sync(FULL, mbar_wait(acc_empty + ab, ((u >> 1) - 1) & 1, wc, kErrWaitMma));
           if (!ok) break;
         }
         tc_fence_after();
@@ -177,16 +217,18 @@ __global__ void __launch_bounds__(256, 1)
         if (lane == 0) {
           const uint32_t idesc = idesc_bf16_f32(128, nc, 0, 0);
           const uint32_t ka = smem_u32(sK + slot * S::kKTileBytes);
-          const uint32_t qa = smem_u32(sQ + b * S::kQBufBytes);
+          const uint32_t qa = smem_u32(sQ + qb * p.q_buf_bytes);
           const uint32_t qhalf = static_cast<uint32_t>(p.chunk_tokens * G * 128);
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
             const uint32_t qoff = (kk >> 2) * qhalf + (kk & 3) * 32;
-            mma_ss(tmem + b * 256, sdesc_sw128(ka + koff, 16, 1024), sdesc_sw128(qa + qoff, 16, 1024), idesc,
+            mma_ss(tmem + ab * 256, sdesc_sw128(ka + koff, 16, 1024), sdesc_sw128(qa + qoff, 16, 1024), idesc,
                    kk > 0 ? 1u : 0u);
           }
-          mma_commit(acc_full + b);
-          if (u + 2 < total_uses && score_needs_load(p, first, u + 2)) mma_commit(q_empty + b);
+          mma_commit(acc_full + ab);
+          int ln, cn;
+          score_next_use(p, li, c, &ln, &cn);
+          if (ln < n_local && score_needs_load(p, s_items, ln, cn)) mma_commit(q_empty + qb);
         }
         issued_any = true;
         __syncwarp();
@@ -194,6 +236,10 @@ __global__ void __launch_bounds__(256, 1)
       if (!ok) break;
       if (lane == 0) mma_commit(k_empty + slot);
       __syncwarp();
+      if (++slot == n_stages) {
+        slot = 0;
+        kphase ^= 1;
+      }
     }
     if (issued_any) {
       if (lane == 0) {
@@ -209,7 +255,7 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     bool ok = true;
     for (int li = 0; li < n_local && ok; ++li) {
-      const int4 it = __ldg(p.items + first + li);
+      const int4 it = s_items[li];
       const int j = it.z + row;  // key position
       const int e = it.w;
       float mx = -INFINITY;
@@ -223,17 +269,32 @@ __global__ void __launch_bounds__(256, 1)
         // Column n is probe token c*Rc + n/G, i.e. row e - R + c*Rc + n/G; it may score
         // key j iff that row >= j, i.e. n >= G * (j - (e - R + c*Rc)).
         const int col_min = G * (j - (e - p.probe_r + c * p.chunk_tokens));
-        for (int n0 = 0; n0 < nc; n0 += 16) {
+        int n0 = 0;
+        // Whole 128-column blocks: one TMEM load each, then a three-input max tree.
+        for (; n0 + 128 <= nc; n0 += 128) {
+          uint32_t v[128];
+          tmem_ld_x128(tl + b * 256 + n0, v);
+          if (col_min > n0) {
+#pragma unroll
+            for (int t = 0; t < 128; ++t)
+              if (n0 + t < col_min) v[t] = 0xff800000u;  // -inf: probe row before key j
+          }
+          float m8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) m8[k] = fmaxf(__uint_as_float(v[k]), __uint_as_float(v[k + 8]));
+#pragma unroll
+          for (int t = 16; t < 128; t += 16)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], __uint_as_float(v[t + k]), __uint_as_float(v[t + 8 + k]));
+          mx = fmax3(mx, fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])), -INFINITY);
+        }
+        // Remaining columns (chunks that are not a multiple of 128) in 16-column loads.
+        for (; n0 < nc; n0 += 16) {
           uint32_t v[16];
           tmem_ld_x16(tl + b * 256 + n0, v);
-          if (col_min <= n0) {
 #pragma unroll
-            for (int t = 0; t < 16; ++t) mx = fmaxf(mx, __uint_as_float(v[t]));
-          } else {
-#pragma unroll
-            for (int t = 0; t < 16; ++t)
-              if (n0 + t >= col_min) mx = fmaxf(mx, __uint_as_float(v[t]));
-          }
+          for (int t = 0; t < 16; ++t)
+            if (n0 + t >= col_min) mx = fmaxf(mx, __uint_as_float(v[t]));
         }
         tc_fence_before();
         __syncwarp();

@@ -50,9 +50,24 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
 // P-th largest key T and how many keys equal to T are taken; a stable compaction in
 // index order then writes the P winners ascending: keys > T, and the lowest-index
 // keys == T.  Result is bit-exact and independent of thread timing.
+// Thread t owns the contiguous keys [t*per, (t+1)*per).  With kPer > 0 they are read
+// once into registers (segments up to kPer * blockDim.x keys); kPer == 0 re-reads
+// them from global memory on every pass (any segment length).
+// With kGather the CTA then copies its P passing rows of K and V into
+// k_pass/v_pass[g][h] (16 bytes per thread), so the prefill needs no separate gather.
+struct GatherArgs {
+  const uint4* k;
+  const uint4* v;
+  uint4* kp;
+  uint4* vp;
+  int hosts_m1;
+  int chunks_per_row;  // 16-byte chunks per K/V row (d * 2 / 16)
+};
+
+template <int kPer, bool kGather>
 __global__ void __launch_bounds__(1024) select_topp_kernel(const float* __restrict__ scores, int n_visual,
                                                             const int* __restrict__ off, int anchor, int passing,
-                                                            int hkv, int32_t* __restrict__ idx) {
+                                                            int hkv, int32_t* __restrict__ idx, GatherArgs ga) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t scan_scratch[33];
   __shared__ uint32_t sh_prefix, sh_k;
@@ -63,14 +78,28 @@ __global__ void __launch_bounds__(1024) select_topp_kernel(const float* __restri
   int32_t* out = idx + (static_cast<size_t>(h) * hkv + g) * passing;
   const int tid = threadIdx.x, nt = blockDim.x;
   if (passing <= 0) return;
+  const int per = (n + nt - 1) / nt;
+  const int j0 = min(n, tid * per), cnt = min(n, j0 + per) - j0;
+
+  constexpr int kRegs = kPer > 0 ? kPer : 1;
+  uint32_t u[kRegs];
+  if (kPer > 0) {
+#pragma unroll
+    for (int i = 0; i < kRegs; ++i) u[i] = i < cnt ? ordered_key(__ldg(s + j0 + i)) : 0u;
+  }
+  auto key = [&](int i) -> uint32_t { return kPer > 0 ? u[i] : ordered_key(__ldg(s + j0 + i)); };
+  const int n_loop = kPer > 0 ? kRegs : per;
 
   uint32_t prefix = 0u, pmask = 0u, k = static_cast<uint32_t>(passing);
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int t = tid; t < 256; t += nt) hist[t] = 0u;
     __syncthreads();
-    for (int j = tid; j < n; j += nt) {
-      const uint32_t u = ordered_key(__ldg(s + j));
-      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 0xFFu], 1u);
+#pragma unroll
+    for (int i = 0; i < n_loop; ++i) {
+      if (i < cnt) {
+        const uint32_t x = key(i);
+        if ((x & pmask) == prefix) atomicAdd(&hist[(x >> shift) & 0xFFu], 1u);
+      }
     }
     __syncthreads();
     if (tid < 32) {
@@ -105,32 +134,46 @@ __global__ void __launch_bounds__(1024) select_topp_kernel(const float* __restri
     prefix = sh_prefix;
     k = sh_k;
     pmask |= 0xFFu << shift;
-    __syncthreads();
   }
-  const uint32_t T = prefix;       // key of the P-th largest score
-  const uint32_t take_eq = k;      // keys equal to T that are selected (lowest index first)
+  const uint32_t T = prefix;   // key of the P-th largest score
+  const uint32_t take_eq = k;  // keys equal to T that are selected (lowest index first)
 
-  // Stable compaction: thread t owns keys [t*per, (t+1)*per).
-  const int per = (n + nt - 1) / nt;
-  const int j0 = min(n, tid * per), j1 = min(n, j0 + per);
   uint32_t cgt = 0u, ceq = 0u;
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t u = ordered_key(__ldg(s + j));
-    cgt += u > T;
-    ceq += u == T;
+#pragma unroll
+  for (int i = 0; i < n_loop; ++i) {
+    if (i < cnt) {
+      const uint32_t x = key(i);
+      cgt += x > T;
+      ceq += x == T;
+    }
   }
   uint32_t tot;
   const uint32_t eq_before = block_exclusive_scan(ceq, scan_scratch, &tot);
   const uint32_t eq_take = eq_before >= take_eq ? 0u : min(ceq, take_eq - eq_before);
   uint32_t pos = block_exclusive_scan(cgt + eq_take, scan_scratch, &tot);
   uint32_t eq_seen = eq_before;
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t u = ordered_key(__ldg(s + j));
-    if (u > T) {
-      out[pos++] = lo + j;
-    } else if (u == T) {
-      if (eq_seen < take_eq) out[pos++] = lo + j;
-      ++eq_seen;
+#pragma unroll
+  for (int i = 0; i < n_loop; ++i) {
+    if (i < cnt) {
+      const uint32_t x = key(i);
+      if (x > T) {
+        out[pos++] = lo + j0 + i;
+      } else if (x == T) {
+        if (eq_seen < take_eq) out[pos++] = lo + j0 + i;
+        ++eq_seen;
+      }
+    }
+  }
+  if (kGather) {
+    __syncthreads();  // the block's index writes are visible to the block after this
+    const int cpr = ga.chunks_per_row;
+    const size_t dst0 = ((static_cast<size_t>(g) * ga.hosts_m1 + h) * passing) * cpr;
+    for (int t = tid; t < passing * cpr; t += nt) {
+      const int r = t / cpr, ch = t - r * cpr;
+      const int tok = out[r];
+      const size_t src = (static_cast<size_t>(tok) * hkv + g) * cpr + ch;
+      ga.kp[dst0 + t] = __ldg(ga.k + src);
+      ga.vp[dst0 + t] = __ldg(ga.v + src);
     }
   }
 }

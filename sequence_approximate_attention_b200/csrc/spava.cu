@@ -3,8 +3,9 @@
 //
 // Call graph of spava_attn_prefill, all on the caller's stream:
 //   score_kernel      probe scores of hosts 0..H-2 (tensor cores)
-//   select_topp       top-P passing keys per (host, KV head)
-//   gather_passing    passing K/V into one contiguous buffer per KV head
+//   select_topp       top-P passing keys per (host, KV head), each CTA then
+//                     gathering its passing K/V rows into one contiguous buffer
+//                     per KV head (spava_gather_passing runs that gather alone)
 //   attn_fwd_kernel   one flash-attention pass per host item, text rows as
 //                     split-KV partials over the host blocks
 //   lse_merge         text partials -> final rows
@@ -127,7 +128,9 @@ namespace {
 
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-enum KernelLabel { kLabScore = 0, kLabSelect = 1, kLabGather = 2, kLabAttn = 3, kLabMerge = 4, kLabDense = 5 };
+enum KernelLabel {
+  kLabScore = 0, kLabSelect = 1, kLabGather = 2, kLabAttn = 3, kLabMerge = 4, kLabDense = 5, kLabSelectGather = 6
+};
 
 void mark(const spava_plan* p, int label, cudaStream_t st) {
   if (p->prof_used >= static_cast<int>(p->prof_ev.size())) return;
@@ -258,19 +261,48 @@ spava_status launch_score(const spava_plan* p, const void* q, const void* k, flo
   sp.err_word = err_word(p, ws);
   sp.wait_limit_ns = p->wait_limit_ns;
   using S = spava::ScoreShape<D>;
-  if ((s = ensure_smem(spava::score_kernel<D>, S::kSmemBytes)) != SPAVA_OK) return s;
-  const int grid = std::min(n_items, p->num_sms);
+  // Probe-query buffers: one when every (host, group) is a single chunk (it stays
+  // resident across that group's key tiles), two otherwise; the rest of shared
+  // memory holds K-tile stages.
+  sp.q_bufs = p->n_chunks == 1 ? 1 : 2;
+  sp.q_buf_bytes = (D / 64) * p->rc * G * 128;
+  sp.k_stages = std::min<int>(S::kMaxStages, (S::kSmemMax - S::smem_bytes(sp.q_bufs, sp.q_buf_bytes, 0)) / S::kKTileBytes);
+  if (sp.k_stages < 2) return fail(SPAVA_ERR_UNSUPPORTED, "probe queries too large for shared memory");
+  const int smem = S::smem_bytes(sp.q_bufs, sp.q_buf_bytes, sp.k_stages);
+  if ((s = ensure_smem(spava::score_kernel<D>, S::kSmemMax)) != SPAVA_OK) return s;
+  int grid = std::min(n_items, p->num_sms);
+  // every CTA's item range must fit the kernel's shared-memory item cache
+  grid = std::max(grid, (n_items + S::kMaxLocalItems - 1) / S::kMaxLocalItems);
   mark(p, kLabScore, st);
-  spava::score_kernel<D><<<grid, 256, S::kSmemBytes, st>>>(tmK, tmQp, sp);
+  spava::score_kernel<D><<<grid, 256, smem, st>>>(tmK, tmQp, sp);
   SPAVA_CUDA(cudaGetLastError());
   ++g_last_launches;
   return SPAVA_OK;
 }
 
-spava_status launch_select(const spava_plan* p, const float* scores, int32_t* idx, cudaStream_t st) {
+// Top-P selection; with k/v/kp/vp given, each selection CTA also gathers its passing
+// rows (the prefill's fused select + gather).
+spava_status launch_select(const spava_plan* p, const float* scores, int32_t* idx, cudaStream_t st,
+                           const void* k = nullptr, const void* v = nullptr, void* kp = nullptr, void* vp = nullptr) {
   if (p->H < 2 || p->P == 0) return SPAVA_OK;
-  mark(p, kLabSelect, st);
-  spava::select_topp_kernel<<<(p->H - 1) * p->hkv, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, p->hkv, idx);
+  int max_seg = 0;
+  for (int h = 0; h + 1 < p->H; ++h) max_seg = std::max(max_seg, p->off[h + 1] - p->off[h]);
+  spava::GatherArgs ga{static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(kp),
+                       static_cast<uint4*>(vp), p->H - 1, p->d * 2 / 16};
+  const bool fused = k != nullptr;
+  const int grid = (p->H - 1) * p->hkv;
+  mark(p, fused ? kLabSelectGather : kLabSelect, st);
+  if (max_seg <= 16 * 1024) {
+    if (fused)
+      spava::select_topp_kernel<16, true><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, p->hkv, idx, ga);
+    else
+      spava::select_topp_kernel<16, false><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, p->hkv, idx, ga);
+  } else {
+    if (fused)
+      spava::select_topp_kernel<0, true><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, p->hkv, idx, ga);
+    else
+      spava::select_topp_kernel<0, false><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, p->hkv, idx, ga);
+  }
   SPAVA_CUDA(cudaGetLastError());
   ++g_last_launches;
   return SPAVA_OK;
@@ -588,8 +620,7 @@ spava_status spava_attn_prefill(const spava_plan* p, const void* q, const void* 
   if (p->H >= 2 && p->P > 0) {
     s = p->d == 128 ? launch_score<128>(p, q, k, scores, false, ws, st) : launch_score<64>(p, q, k, scores, false, ws, st);
     if (s != SPAVA_OK) return s;
-    if ((s = launch_select(p, scores, idx, st)) != SPAVA_OK) return s;
-    if ((s = launch_gather(p, k, v, idx, kp, vp, st)) != SPAVA_OK) return s;
+    if ((s = launch_select(p, scores, idx, st, k, v, kp, vp)) != SPAVA_OK) return s;
   }
   s = p->d == 128 ? launch_attn<128>(p, p->d_items_pre, p->n_items_pre, q, k, v, kp, vp, o, lse, ws, st)
                   : launch_attn<64>(p, p->d_items_pre, p->n_items_pre, q, k, v, kp, vp, o, lse, ws, st);
@@ -712,6 +743,7 @@ const char* spava_kernel_name(int32_t label) {
     case kLabAttn: return "attention";
     case kLabMerge: return "lse_merge";
     case kLabDense: return "attention_dense";
+    case kLabSelectGather: return "select_gather";
   }
   return "unknown";
 }
