@@ -66,6 +66,48 @@ def select_gather_bytes(cfg, sizes):
     return {"score": score, "select": select, "gather": gather, "select_gather": select + gather}
 
 
+def attn_algorithmic_bytes(cfg):
+    """DRAM bytes the attention kernel must move once: Q, K, V and the passing K/V
+    read, O (bf16, visual rows) and the text partials (fp32, one per host block plus
+    the causal piece) written, lse written."""
+    NT, N, T, H = cfg.n_visual + cfg.n_text, cfg.n_visual, cfg.n_text, cfg.n_hosts
+    d, hq, hkv, P = cfg.head_dim, cfg.hq, cfg.hkv, cfg.passing
+    rd = NT * hq * d * 2 + 2 * NT * hkv * d * 2 + 2 * hkv * max(H - 1, 0) * P * d * 2
+    wr = N * hq * d * 2 + hq * N * 4 + (H + 1) * T * hq * (d + 1) * 4
+    return rd + wr
+
+
+# The ncu traffic of the attention kernel is recorded in profiles/ together with a
+# digest of the sources it was measured on (kernel and plan ordering); the bench
+# reports it only while that digest still matches, else null.
+TRAFFIC_NOTE = os.path.join(ROOT, "profiles", "attn_fwd_128k_traffic.md")
+TRAFFIC_SOURCES = [os.path.join("sequence_approximate_attention_b200", "csrc", f)
+                   for f in ("attn_kernel.cuh", "common.cuh", "tmem_ops.inc", "exp2_poly.inc", "spava.cu")]
+
+
+def attn_source_digest():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload):
+    import re
+    try:
+        text = open(TRAFFIC_NOTE).read()
+    except OSError:
+        return None
+    w = re.search(r"workload:\s*(\S+)", text)
+    b = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
+    dg = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    if not (w and b and dg) or w.group(1) != workload or dg.group(1) != attn_source_digest():
+        return None
+    return int(b.group(1))
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -74,6 +116,27 @@ def load_peaks():
         return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(value, device=None):
+    """Max of a per-rank float over all ranks of the default process group (the
+    value itself when no group is initialised).  NCCL needs a CUDA device tensor,
+    gloo a CPU one."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, tokens_per_step, steps, ms_max):
+    """Whole-job tokens/s: every rank runs its own replica of the workload (weak
+    scaling), so the job processes world * tokens_per_step * steps tokens in the
+    slowest rank's time."""
+    return world * tokens_per_step * steps / (ms_max / 1e3)
 
 
 # ---------------------------------------------------------------- clocks
@@ -305,12 +368,9 @@ def main():
     prof = plan.profile_read()
     plan.profile_end()
     sab.check_device_error(plan, ws)
-    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / args.steps
-    value = world * NT * args.steps / (ms_total / 1e3)
+    value = job_throughput(world, NT, args.steps, ms_total)
 
     # per-kernel averages over the timed steps
     per = {}
@@ -333,7 +393,8 @@ def main():
     ssg_bytes = sum(sgb[n] for n in ssg_names)
     roofline = {
         "bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved, "peak": peaks["bf16_tflops"],
-        "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+        "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": recorded_traffic(cfg.name),
+        "algorithmic_bytes": attn_algorithmic_bytes(cfg),
         "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)",
         "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
         "frac_of_datasheet_2250": achieved / 2250.0,
@@ -390,10 +451,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * NT * args.e2e_steps / (float(te.item()) / 1e3), "unit": "tokens/s",
+        te = max_over_ranks(e0.elapsed_time(e1), dev)
+        e2e = {"value": job_throughput(world, NT, args.e2e_steps, te), "unit": "tokens/s",
                "h2d_bytes_per_step": sum(pin[x].numel() * 2 for x in pin),
                "d2h_bytes_per_step": o_h.numel() * 2 + l_h.numel() * 4, "steps": args.e2e_steps}
 

@@ -150,6 +150,28 @@ void sort_by_cost(std::vector<AttnItem>& v) {
   std::stable_sort(v.begin(), v.end(), [](const AttnItem& a, const AttnItem& b) { return item_cost(a) > item_cost(b); });
 }
 
+// Prefill order: hosts from the longest KV list to the shortest, KV groups in order
+// inside a host, longest items first inside a group.  Consecutive items (which run
+// at the same time on the 148 CTAs) then share one host's block, the anchor and the
+// passing rows of one or two KV groups, a working set that stays in L2, while every
+// round of CTAs still gets a spread of item costs for balance.
+// `group` gives each item its host (text pieces are grouped with the host block
+// they read, their own causal piece with the last host).
+void sort_host_major(std::vector<AttnItem>& v, const std::vector<int>& group, int heads_per_group) {
+  auto kv_group_of = [&](const AttnItem& it) { return it.q_head / heads_per_group; };
+  std::vector<int> order(v.size());
+  for (size_t i = 0; i < v.size(); ++i) order[i] = static_cast<int>(i);
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+    if (group[a] != group[b]) return group[a] > group[b];
+    if (kv_group_of(v[a]) != kv_group_of(v[b])) return kv_group_of(v[a]) < kv_group_of(v[b]);
+    return item_cost(v[a]) > item_cost(v[b]);
+  });
+  std::vector<AttnItem> out;
+  out.reserve(v.size());
+  for (int i : order) out.push_back(v[i]);
+  v.swap(out);
+}
+
 AttnItem blank_item(int q_row0, int q_rows, int q_head, int slot) {
   AttnItem it;
   std::memset(&it, 0, sizeof(it));
@@ -166,6 +188,7 @@ AttnItem blank_item(int q_row0, int q_rows, int q_head, int slot) {
 // piece writing an fp32 partial with its lse.
 std::vector<AttnItem> build_prefill_items(const spava_plan& p) {
   std::vector<AttnItem> v;
+  std::vector<int> group;
   for (int h = 0; h < p.H; ++h) {
     const int a = p.off[h], e = p.off[h + 1];
     for (int r0 = a; r0 < e; r0 += 256) {
@@ -177,6 +200,7 @@ std::vector<AttnItem> build_prefill_items(const spava_plan& p) {
         if (h >= 1 && p.P > 0) it.seg[ns++] = AttnSeg{0, h * p.P, spava::kSegPassing, 0};
         it.seg[ns++] = AttnSeg{a, r0 + rows - a, spava::kSegCausal, 0};
         v.push_back(it);
+        group.push_back(h);
       }
     }
   }
@@ -190,10 +214,11 @@ std::vector<AttnItem> build_prefill_items(const spava_plan& p) {
         else
           it.seg[0] = AttnSeg{p.N, r0 + rows - p.N, spava::kSegCausal, 0};
         v.push_back(it);
+        group.push_back(k < p.H ? k : p.H - 1);
       }
     }
   }
-  sort_by_cost(v);
+  sort_host_major(v, group, p.hq / p.hkv);
   return v;
 }
 
