@@ -182,6 +182,35 @@ spava_status spava_attn_prefill_noalloc(const spava_plan* plan, const void* q, c
                                         const void* v, void* o, float* lse, void* stream);
 
 /*
+ * The same prefill in the two stages the pages describe (APB-V technical summary,
+ * "Main contributions": two-stage attention; 1. Framework design: passing blocks
+ * picked by query-to-context scores; 2. System optimisations: partial results merged
+ * through FlashAttention's lse):
+ *   stage 1  every host's queries over its own block, causal, on the attention
+ *            kernel; the items that hold a host's last R query rows fold their raw
+ *            q.k logits into the probe scores as they go (fused scoring: column
+ *            maxima per warp, max over the group's query heads by atomic max on
+ *            order-preserving integer keys); hosts with a remote part keep fp32
+ *            partial O and lse of their rows;
+ *   select + gather of the passing rows;
+ *   stage 2  host h >= 1 over [anchor | passing of hosts < h], merged with its
+ *            stage-1 partial through the lse into the final O and lse;
+ *   text rows as in spava_attn_prefill.
+ * Arguments and layouts as spava_attn_prefill; `ws` must hold
+ * spava_two_stage_workspace_bytes(plan) bytes (it adds the fp32 row partials,
+ * N * hq * d * 4 bytes).  Results equal spava_attn_prefill's up to fp32 rounding
+ * order (the scores come from a different MMA, so selections may differ at exact
+ * ties within rounding).  spava_attn_prefill is the faster flow on one GPU: it needs
+ * no partials of the visual rows.
+ */
+spava_status spava_attn_prefill_two_stage(const spava_plan* plan, const void* q, const void* k,
+                                          const void* v, void* o, float* lse, float* scores_out,
+                                          int32_t* idx_out, void* ws, void* stream);
+
+/* Workspace bytes of spava_attn_prefill_two_stage (0 if plan is NULL). */
+size_t spava_two_stage_workspace_bytes(const spava_plan* plan);
+
+/*
  * Dense causal attention over all N+T tokens on the same kernel (the standard
  * FlashAttention the method degenerates to on one host; the comparison kernel).
  * Layouts as above.
@@ -213,7 +242,8 @@ int32_t spava_profile_read(spava_plan* plan, int32_t* labels, float* ms, int32_t
 spava_status spava_profile_end(spava_plan* plan);
 
 /* Name of a kernel label: 0 score, 1 select, 2 gather, 3 attention (prefill),
- * 4 lse merge, 5 attention (dense causal), 6 select + gather (fused, prefill). */
+ * 4 lse merge, 5 attention (dense causal), 6 select + gather (fused, prefill),
+ * 7 score-key fill/convert (two-stage), 8 attention stage 1, 9 attention stage 2. */
 const char* spava_kernel_name(int32_t label);
 
 /* Static text of a status code. */

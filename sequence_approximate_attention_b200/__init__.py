@@ -18,7 +18,7 @@ import torch
 from . import _lib
 from ._lib import SpavaError, load  # noqa: F401
 
-__all__ = ["Plan", "score_select", "gather_passing", "attn_prefill", "dense_causal",
+__all__ = ["Plan", "score_select", "gather_passing", "attn_prefill", "attn_prefill_two_stage", "dense_causal",
            "check_device_error", "SpavaError", "load", "last_launch_count"]
 
 
@@ -69,6 +69,7 @@ class Plan:
         _lib.check(st, "spava_plan_create")
         self._h = handle
         self.workspace_bytes = int(self.lib.spava_workspace_bytes(self._h))
+        self.two_stage_workspace_bytes = int(self.lib.spava_two_stage_workspace_bytes(self._h))
         off = (ctypes.c_int32 * (self.n_hosts + 1))()
         self.lib.spava_plan_offsets(self._h, off)
         self.offsets = [int(x) for x in off]
@@ -81,8 +82,9 @@ class Plan:
     def n_total(self) -> int:
         return self.n_visual + self.n_text
 
-    def new_workspace(self) -> torch.Tensor:
-        return torch.zeros(max(self.workspace_bytes, 256), dtype=torch.uint8, device=self.device)
+    def new_workspace(self, two_stage: bool = False) -> torch.Tensor:
+        n = self.two_stage_workspace_bytes if two_stage else self.workspace_bytes
+        return torch.zeros(max(n, 256), dtype=torch.uint8, device=self.device)
 
     def set_debug(self, wait_limit_ns: int = 0, stall_producer: bool = False) -> None:
         _lib.check(self.lib.spava_plan_set_debug(self._h, int(wait_limit_ns), int(bool(stall_producer))),
@@ -134,12 +136,13 @@ class Plan:
             _expect(v, "v", torch.bfloat16, ks, self.device)
 
 
-def _ws(plan: Plan, workspace: Optional[torch.Tensor]) -> torch.Tensor:
+def _ws(plan: Plan, workspace: Optional[torch.Tensor], two_stage: bool = False) -> torch.Tensor:
     if workspace is None:
-        workspace = plan.new_workspace()
-    if workspace.dtype != torch.uint8 or workspace.numel() < plan.workspace_bytes or \
+        workspace = plan.new_workspace(two_stage)
+    need = plan.two_stage_workspace_bytes if two_stage else plan.workspace_bytes
+    if workspace.dtype != torch.uint8 or workspace.numel() < need or \
             workspace.device != plan.device or workspace.data_ptr() % 256:
-        raise ValueError("workspace: uint8, 256-byte aligned, >= plan.workspace_bytes on the plan's device")
+        raise ValueError(f"workspace: uint8, 256-byte aligned, >= {need} bytes on the plan's device")
     return workspace
 
 
@@ -209,6 +212,32 @@ def attn_prefill(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     st = plan.lib.spava_attn_prefill(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                                      _ptr(scores_out), _ptr(idx_out), _ptr(ws), _stream(stream))
     _lib.check(st, "spava_attn_prefill")
+    return o, lse
+
+
+def attn_prefill_two_stage(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                           o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                           scores_out: Optional[torch.Tensor] = None, idx_out: Optional[torch.Tensor] = None,
+                           workspace: Optional[torch.Tensor] = None, stream=None):
+    """spava_attn_prefill_two_stage: the prefill as local pass (with fused probe scores)
+    -> select/gather -> remote pass merged through the lse.  Needs the larger
+    plan.two_stage_workspace_bytes workspace."""
+    plan._check_qkv(q, k, v)
+    dev = plan.device
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((plan.hq, plan.n_total), dtype=torch.float32, device=dev)
+    _expect(o, "o", torch.bfloat16, tuple(q.shape), dev)
+    _expect(lse, "lse", torch.float32, (plan.hq, plan.n_total), dev)
+    if scores_out is not None:
+        _expect(scores_out, "scores_out", torch.float32, (plan.hkv, plan.n_visual), dev)
+    if idx_out is not None:
+        _expect(idx_out, "idx_out", torch.int32, plan.idx_shape(), dev)
+    ws = _ws(plan, workspace, two_stage=True)
+    st = plan.lib.spava_attn_prefill_two_stage(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                               _ptr(scores_out), _ptr(idx_out), _ptr(ws), _stream(stream))
+    _lib.check(st, "spava_attn_prefill_two_stage")
     return o, lse
 
 

@@ -32,6 +32,9 @@ SIGNATURES = {
                                      c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "spava_attn_prefill_noalloc": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                              c_void_p, c_void_p]),
+    "spava_attn_prefill_two_stage": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                               c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "spava_two_stage_workspace_bytes": (c_size_t, [c_void_p]),
     "spava_dense_causal": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                      c_void_p, c_void_p, c_void_p]),
     "spava_check_device_error": (c_int32, [c_void_p, c_void_p, c_void_p]),

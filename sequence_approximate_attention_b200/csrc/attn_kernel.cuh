@@ -38,14 +38,27 @@ struct AttnSeg {
   int row0;   // first row (token position, or row of the passing buffer)
   int len;    // rows in the segment (0 = unused)
   int flags;  // kSegCausal | kSegPassing
-  int pad;
+  int aux;    // causal segment of a scoring item: end of the host block
 };
 
+// What an item does with its result (bits 24..27 of AttnItem::out), plus a flag that
+// makes it also contribute probe scores (two-stage flow) and a partial slot.
+enum : int {
+  kOutFinal = 0,        // bf16 O and lse of these rows
+  kOutTextPartial = 1,  // fp32 partial O and lse into text slot (out & 0xFFFF)
+  kOutRowPartial = 2,   // fp32 partial O and lse of visual rows (local pass)
+  kOutMerge = 3,        // lse-merge with the rows' partial, then bf16 O and lse
+};
+constexpr int kOutScore = 1 << 20;
+__host__ __device__ constexpr int make_out(int mode, int slot = 0, bool score = false) {
+  return (mode << 24) | (score ? kOutScore : 0) | slot;
+}
+
 struct AttnItem {
-  int q_row0;    // first query row (token position)
-  int q_rows;    // 1..256 valid query rows
-  int q_head;    // query head
-  int out_slot;  // < 0: final bf16 output; >= 0: fp32 partial slot
+  int q_row0;  // first query row (token position)
+  int q_rows;  // 1..256 valid query rows
+  int q_head;  // query head
+  int out;     // make_out(mode, slot, score)
   AttnSeg seg[3];
 };
 static_assert(sizeof(AttnItem) == 64, "AttnItem layout");
@@ -66,6 +79,13 @@ struct AttnParams {
   unsigned int* err_word;
   uint64_t wait_limit_ns;
   int stall_producer;
+  // two-stage flow
+  float* row_o;               // [N][hq][D] fp32 partials of visual rows
+  float* row_lse;             // [hq][N]
+  unsigned int* score_keys;   // [hkv][N] ordered probe-score keys, max-reduced
+  int n_visual;
+  int probe_r;
+  float scale;                // softmax scale (scores are max(q.k) * scale)
 };
 
 // Pairs (out of every 8) whose exp2 runs on the FMA/ALU pipes (exp2_poly2) instead
@@ -106,7 +126,7 @@ __device__ __forceinline__ AttnSeg seg_at(const AttnItem& it, int s) {
   r.row0 = s == 0 ? it.seg[0].row0 : (s == 1 ? it.seg[1].row0 : it.seg[2].row0);
   r.len = s == 0 ? it.seg[0].len : (s == 1 ? it.seg[1].len : it.seg[2].len);
   r.flags = s == 0 ? it.seg[0].flags : (s == 1 ? it.seg[1].flags : it.seg[2].flags);
-  r.pad = 0;
+  r.aux = s == 0 ? it.seg[0].aux : (s == 1 ? it.seg[1].aux : it.seg[2].aux);
   return r;
 }
 
@@ -130,6 +150,24 @@ struct TileCursor {
   }
   __device__ __forceinline__ bool done() const { return s >= 3; }
 };
+
+// Column maxima of a warp's 32 rows x 32 columns (v: this lane's row) by recursive
+// halving: at each step a lane keeps one half of its columns and sends the other to
+// the partner lane (xor 16, 8, 4, 2, 1); 31 shuffles.  On return lane l holds the
+// maximum of column l in v[0].
+__device__ __forceinline__ void warp_column_max32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int s = 0; s < 5; ++s) {
+    const int half = 16 >> s, mask = 16 >> s;
+    const bool upper = (lane & mask) != 0;
+#pragma unroll
+    for (int k = 0; k < half; ++k) {
+      const float keep = upper ? v[k + half] : v[k];
+      const float send = upper ? v[k] : v[k + half];
+      v[k] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, mask));
+    }
+  }
+}
 
 // Static longest-first schedule: items are sorted by cost (descending); CTA b takes
 // item r*G + b in even rounds and r*G + G-1-b in odd rounds (snake order).
@@ -411,6 +449,8 @@ __global__ void __launch_bounds__(384, 1)
       if (i == 1 && it.q_rows <= 128) continue;
       const int qrow0 = it.q_row0 + i * 128;
       const int qpos = qrow0 + row;
+      const int out_mode = (it.out >> 24) & 0xF;
+      const bool score_item = (it.out & kOutScore) != 0;
       float m_run = -INFINITY, l_run = 0.f;
       int j = 0;
       TileCursor cur;
@@ -469,6 +509,29 @@ __global__ void __launch_bounds__(384, 1)
         }
         const float2 r01 = fadd2(rs[0], rs[1]), r23 = fadd2(rs[2], rs[3]), r = fadd2(r01, r23);
         l_run = l_run * alpha + (r.x + r.y);
+        if (score_item && causal) {
+          // Two-stage flow: this item holds probe rows [aux - R, aux) of its host; fold
+          // their raw q.k into the per-key scores (max over probe rows here, over the
+          // group's query heads through the atomic max).  S is still intact in TMEM
+          // (P has not been stored yet) and is re-read 32 columns at a time.
+          const bool probe_row = qpos >= sg.aux - p.probe_r && qpos < sg.aux && (i * 128 + row) < it.q_rows;
+          if (__any_sync(FULL, probe_row)) {
+            unsigned int* keys = p.score_keys + static_cast<size_t>(it.q_head / p.group) * p.n_visual + kpos0;
+            int lim = valid;
+            if (causal) lim = min(lim, qpos - kpos0 + 1);
+#pragma unroll 1
+            for (int h0 = 0; h0 < 128; h0 += 32) {
+              uint32_t raw[32];
+              tmem_ld_x32(tl + S::tmem_s(i) + h0, raw);
+              float cv[32];
+#pragma unroll
+              for (int c = 0; c < 32; ++c) cv[c] = (probe_row && h0 + c < lim) ? __uint_as_float(raw[c]) : -INFINITY;
+              warp_column_max32(cv, lane);
+              const int c = h0 + lane;
+              if (c < valid && cv[0] != -INFINITY) atomicMax(keys + c, ordered_key(cv[0] * p.scale));
+            }
+          }
+        }
         tmem_st_x64(tl + S::tmem_s(i), *reinterpret_cast<uint32_t(*)[64]>(sr));
         if (rescale) {
           // O_i holds the sum up to tile j-1 (its MMA finished before S_i(j) did).
@@ -494,29 +557,66 @@ __global__ void __launch_bounds__(384, 1)
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.0f;
       const bool store = (i * 128 + row) < it.q_rows;
       const int grow = qpos;
-      if (it.out_slot < 0) {
+      const float lse_own = (m_use + log2f(l_run)) * 0.69314718055994531f;
+      if (out_mode == kOutFinal || out_mode == kOutMerge) {
+        // kOutMerge: combine with the rows' local partial through the lse.
+        float w_own = inv_l, w_loc = 0.f, lse_out = lse_own;
+        const float* lrow = nullptr;
+        if (out_mode == kOutMerge) {
+          const float lse_loc = p.row_lse[static_cast<size_t>(it.q_head) * p.n_visual + grow];
+          const float mm = fmaxf(lse_loc, lse_own);
+          const float e_loc = expf(lse_loc - mm), e_own = expf(lse_own - mm);
+          lse_out = mm + logf(e_loc + e_own);
+          const float inv = 1.0f / (e_loc + e_own);
+          w_own = inv_l * e_own * inv;
+          w_loc = e_loc * inv;
+          lrow = p.row_o + (static_cast<size_t>(grow) * p.hq + it.q_head) * D;
+        }
         __nv_bfloat16* orow = p.o + (static_cast<size_t>(grow) * p.hq + it.q_head) * D;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t ov[32];
           tmem_ld_x32(tl + S::tmem_o(i) + c0, ov);
           if (store) {
+            float f[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) f[c] = __uint_as_float(ov[c]) * w_own;
+            if (out_mode == kOutMerge) {
+              const float4* src = reinterpret_cast<const float4*>(lrow + c0);
+#pragma unroll
+              for (int v4 = 0; v4 < 8; ++v4) {
+                const float4 x = src[v4];
+                f[4 * v4 + 0] = fmaf(x.x, w_loc, f[4 * v4 + 0]);
+                f[4 * v4 + 1] = fmaf(x.y, w_loc, f[4 * v4 + 1]);
+                f[4 * v4 + 2] = fmaf(x.z, w_loc, f[4 * v4 + 2]);
+                f[4 * v4 + 3] = fmaf(x.w, w_loc, f[4 * v4 + 3]);
+              }
+            }
             uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
               uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(ov[8 * v4 + 0]) * inv_l, __uint_as_float(ov[8 * v4 + 1]) * inv_l);
-              w.y = pack_bf16x2(__uint_as_float(ov[8 * v4 + 2]) * inv_l, __uint_as_float(ov[8 * v4 + 3]) * inv_l);
-              w.z = pack_bf16x2(__uint_as_float(ov[8 * v4 + 4]) * inv_l, __uint_as_float(ov[8 * v4 + 5]) * inv_l);
-              w.w = pack_bf16x2(__uint_as_float(ov[8 * v4 + 6]) * inv_l, __uint_as_float(ov[8 * v4 + 7]) * inv_l);
+              w.x = pack_bf16x2(f[8 * v4 + 0], f[8 * v4 + 1]);
+              w.y = pack_bf16x2(f[8 * v4 + 2], f[8 * v4 + 3]);
+              w.z = pack_bf16x2(f[8 * v4 + 4], f[8 * v4 + 5]);
+              w.w = pack_bf16x2(f[8 * v4 + 6], f[8 * v4 + 7]);
               dst[v4] = w;
             }
           }
         }
-        if (store) p.lse[static_cast<size_t>(it.q_head) * p.n_rows_out + grow] = (m_use + log2f(l_run)) * 0.69314718055994531f;
+        if (store) p.lse[static_cast<size_t>(it.q_head) * p.n_rows_out + grow] = lse_out;
       } else {
-        const int prow = grow - p.part_row0;
-        float* orow = p.o_part + ((static_cast<size_t>(it.out_slot) * p.part_rows + prow) * p.hq + it.q_head) * D;
+        // fp32 partials: a text slot, or the visual rows of the local pass
+        float* orow;
+        float* lse_dst;
+        if (out_mode == kOutTextPartial) {
+          const int slot = it.out & 0xFFFF, prow = grow - p.part_row0;
+          orow = p.o_part + ((static_cast<size_t>(slot) * p.part_rows + prow) * p.hq + it.q_head) * D;
+          lse_dst = p.lse_part + (static_cast<size_t>(slot) * p.hq + it.q_head) * p.part_rows + prow;
+        } else {
+          orow = p.row_o + (static_cast<size_t>(grow) * p.hq + it.q_head) * D;
+          lse_dst = p.row_lse + static_cast<size_t>(it.q_head) * p.n_visual + grow;
+        }
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t ov[32];
@@ -529,9 +629,7 @@ __global__ void __launch_bounds__(384, 1)
                                     __uint_as_float(ov[4 * v4 + 2]) * inv_l, __uint_as_float(ov[4 * v4 + 3]) * inv_l);
           }
         }
-        if (store)
-          p.lse_part[(static_cast<size_t>(it.out_slot) * p.hq + it.q_head) * p.part_rows + prow] =
-              (m_use + log2f(l_run)) * 0.69314718055994531f;
+        if (store) *lse_dst = lse_own;
       }
     }
   }

@@ -193,6 +193,19 @@ __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
+// Order-preserving map fp32 -> uint32 (larger float -> larger key).  -0.0 is first
+// made +0.0, so both zeros get the same key.  NaN never reaches here (scores of
+// finite bf16 inputs are finite).
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+  uint32_t b = __float_as_uint(f);
+  if (b == 0x80000000u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+constexpr uint32_t kOrderedNegInf = 0x007fffffu;  // ordered_key(-inf)
+
 // ---------------------------------------------------------------- math helpers
 __device__ __forceinline__ float fast_exp2(float x) {  // MUFU ex2 (ftz); exp2(-inf) = +0
   float y;

@@ -134,7 +134,6 @@ __global__ void __launch_bounds__(256, 1)
   const int first = static_cast<int>((static_cast<long long>(p.n_items) * blockIdx.x) / gridDim.x);
   const int last = static_cast<int>((static_cast<long long>(p.n_items) * (blockIdx.x + 1)) / gridDim.x);
   const int n_local = last - first;
-  const int total_uses = n_local * p.n_chunks;
   const int G = p.group;
   // The host sizes the grid so that every CTA's range fits the shared-memory cache.
   for (int t = threadIdx.x; t < n_local; t += blockDim.x) s_items[t] = __ldg(p.items + first + t);

@@ -6,14 +6,6 @@
 
 namespace spava {
 
-// Order-preserving map fp32 -> uint32 (larger float -> larger key).  -0.0 is first
-// made +0.0, so both zeros get the same key.  NaN never reaches here (scores of
-// finite bf16 inputs are finite).
-__device__ __forceinline__ uint32_t ordered_key(float f) {
-  uint32_t b = __float_as_uint(f);
-  if (b == 0x80000000u) b = 0u;
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
 
 // Exclusive prefix sum over the block (blockDim.x a multiple of 32, <= 1024).
 // `scratch` holds 33 uint32.  Also returns the block total through *total.
@@ -176,6 +168,19 @@ __global__ void __launch_bounds__(1024) select_topp_kernel(const float* __restri
       ga.vp[dst0 + t] = __ldg(ga.v + src);
     }
   }
+}
+
+// Score keys of the two-stage flow: fill with ordered(-inf) before the local pass
+// max-reduces into them, and turn them back into fp32 scores afterwards (in place).
+__global__ void __launch_bounds__(256) fill_u32_kernel(uint32_t* __restrict__ p, size_t n, uint32_t v) {
+  for (size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < n;
+       t += static_cast<size_t>(gridDim.x) * blockDim.x)
+    p[t] = v;
+}
+__global__ void __launch_bounds__(256) keys_to_scores_kernel(uint32_t* __restrict__ p, size_t n) {
+  for (size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < n;
+       t += static_cast<size_t>(gridDim.x) * blockDim.x)
+    p[t] = __float_as_uint(key_to_float(p[t]));
 }
 
 // k_pass[g][h][j][:] = k[idx[h][g][j]][g][:] (same for v), 16 bytes per thread.

@@ -108,12 +108,17 @@ struct spava_plan {
   int n_items_pre = 0;
   AttnItem* d_items_dense = nullptr;
   int n_items_dense = 0;
+  AttnItem* d_items_local = nullptr;   // two-stage flow, first launch
+  int n_items_local = 0;
+  AttnItem* d_items_remote = nullptr;  // two-stage flow, second launch
+  int n_items_remote = 0;
   int4* d_score_pre = nullptr;  // hosts 0..H-2
   int n_score_pre = 0;
   int4* d_score_all = nullptr;  // all hosts
   int n_score_all = 0;
   // workspace layout
   size_t ws_err = 0, ws_scores = 0, ws_idx = 0, ws_kp = 0, ws_vp = 0, ws_opart = 0, ws_lpart = 0, ws_total = 0;
+  size_t ws_row_o = 0, ws_row_lse = 0, ws_total_two_stage = 0;  // two-stage flow only
   // debug knobs
   uint64_t wait_limit_ns = spava::kDefaultWaitLimitNs;
   int stall_producer = 0;
@@ -129,7 +134,8 @@ namespace {
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 enum KernelLabel {
-  kLabScore = 0, kLabSelect = 1, kLabGather = 2, kLabAttn = 3, kLabMerge = 4, kLabDense = 5, kLabSelectGather = 6
+  kLabScore = 0, kLabSelect = 1, kLabGather = 2, kLabAttn = 3, kLabMerge = 4, kLabDense = 5, kLabSelectGather = 6,
+  kLabFill = 7, kLabAttnLocal = 8, kLabAttnRemote = 9
 };
 
 void mark(const spava_plan* p, int label, cudaStream_t st) {
@@ -172,14 +178,33 @@ void sort_host_major(std::vector<AttnItem>& v, const std::vector<int>& group, in
   v.swap(out);
 }
 
-AttnItem blank_item(int q_row0, int q_rows, int q_head, int slot) {
+AttnItem blank_item(int q_row0, int q_rows, int q_head, int out) {
   AttnItem it;
   std::memset(&it, 0, sizeof(it));
   it.q_row0 = q_row0;
   it.q_rows = q_rows;
   it.q_head = q_head;
-  it.out_slot = slot;
+  it.out = out;
   return it;
+}
+
+// Text-query pieces of the prefill (shared by both flows): T rows in 256-row items,
+// split over the host blocks plus their own causal part, each an fp32 partial.
+void add_text_items(const spava_plan& p, std::vector<AttnItem>& v, std::vector<int>& group) {
+  for (int r0 = p.N; r0 < p.N + p.T; r0 += 256) {
+    const int rows = std::min(256, p.N + p.T - r0);
+    for (int c = 0; c < p.hq; ++c) {
+      for (int k = 0; k <= p.H; ++k) {
+        AttnItem it = blank_item(r0, rows, c, spava::make_out(spava::kOutTextPartial, k));
+        if (k < p.H)
+          it.seg[0] = AttnSeg{p.off[k], p.off[k + 1] - p.off[k], 0, 0};
+        else
+          it.seg[0] = AttnSeg{p.N, r0 + rows - p.N, spava::kSegCausal, 0};
+        v.push_back(it);
+        group.push_back(k < p.H ? k : p.H - 1);
+      }
+    }
+  }
 }
 
 // Work list of the prefill.  Host h's rows go in 256-row items per query head with
@@ -194,7 +219,7 @@ std::vector<AttnItem> build_prefill_items(const spava_plan& p) {
     for (int r0 = a; r0 < e; r0 += 256) {
       const int rows = std::min(256, e - r0);
       for (int c = 0; c < p.hq; ++c) {
-        AttnItem it = blank_item(r0, rows, c, -1);
+        AttnItem it = blank_item(r0, rows, c, spava::make_out(spava::kOutFinal));
         int ns = 0;
         if (h >= 1 && p.A > 0) it.seg[ns++] = AttnSeg{0, p.A, 0, 0};
         if (h >= 1 && p.P > 0) it.seg[ns++] = AttnSeg{0, h * p.P, spava::kSegPassing, 0};
@@ -204,17 +229,57 @@ std::vector<AttnItem> build_prefill_items(const spava_plan& p) {
       }
     }
   }
-  for (int r0 = p.N; r0 < p.N + p.T; r0 += 256) {
-    const int rows = std::min(256, p.N + p.T - r0);
-    for (int c = 0; c < p.hq; ++c) {
-      for (int k = 0; k <= p.H; ++k) {
-        AttnItem it = blank_item(r0, rows, c, k);
-        if (k < p.H)
-          it.seg[0] = AttnSeg{p.off[k], p.off[k + 1] - p.off[k], 0, 0};
-        else
-          it.seg[0] = AttnSeg{p.N, r0 + rows - p.N, spava::kSegCausal, 0};
+  add_text_items(p, v, group);
+  sort_host_major(v, group, p.hq / p.hkv);
+  return v;
+}
+
+bool has_remote(const spava_plan& p, int h) { return h >= 1 && (p.A > 0 || p.P > 0); }
+bool scores_needed(const spava_plan& p) { return p.H >= 2 && p.P > 0; }
+
+// Two-stage flow, first launch: every host's queries over its own block (causal).
+// Hosts with a remote part write fp32 partials of their rows; items holding probe
+// rows of hosts < H-1 also fold their logits into the probe scores.  Text pieces
+// run here too.
+std::vector<AttnItem> build_local_items(const spava_plan& p) {
+  std::vector<AttnItem> v;
+  std::vector<int> group;
+  for (int h = 0; h < p.H; ++h) {
+    const int a = p.off[h], e = p.off[h + 1];
+    for (int r0 = a; r0 < e; r0 += 256) {
+      const int rows = std::min(256, e - r0);
+      const bool probe = scores_needed(p) && h < p.H - 1 && r0 + rows > e - p.R;
+      const int mode = has_remote(p, h) ? spava::kOutRowPartial : spava::kOutFinal;
+      for (int c = 0; c < p.hq; ++c) {
+        AttnItem it = blank_item(r0, rows, c, spava::make_out(mode, 0, probe));
+        it.seg[0] = AttnSeg{a, r0 + rows - a, spava::kSegCausal, e};
         v.push_back(it);
-        group.push_back(k < p.H ? k : p.H - 1);
+        group.push_back(h);
+      }
+    }
+  }
+  add_text_items(p, v, group);
+  sort_host_major(v, group, p.hq / p.hkv);
+  return v;
+}
+
+// Two-stage flow, second launch: host h >= 1 over [anchor | passing of hosts < h],
+// lse-merged with its local partial into the final output.
+std::vector<AttnItem> build_remote_items(const spava_plan& p) {
+  std::vector<AttnItem> v;
+  std::vector<int> group;
+  for (int h = 1; h < p.H; ++h) {
+    if (!has_remote(p, h)) continue;
+    const int a = p.off[h], e = p.off[h + 1];
+    for (int r0 = a; r0 < e; r0 += 256) {
+      const int rows = std::min(256, e - r0);
+      for (int c = 0; c < p.hq; ++c) {
+        AttnItem it = blank_item(r0, rows, c, spava::make_out(spava::kOutMerge));
+        int ns = 0;
+        if (p.A > 0) it.seg[ns++] = AttnSeg{0, p.A, 0, 0};
+        if (p.P > 0) it.seg[ns++] = AttnSeg{0, h * p.P, spava::kSegPassing, 0};
+        v.push_back(it);
+        group.push_back(h);
       }
     }
   }
@@ -228,7 +293,7 @@ std::vector<AttnItem> build_dense_items(const spava_plan& p) {
   for (int r0 = 0; r0 < NT; r0 += 256) {
     const int rows = std::min(256, NT - r0);
     for (int c = 0; c < p.hq; ++c) {
-      AttnItem it = blank_item(r0, rows, c, -1);
+      AttnItem it = blank_item(r0, rows, c, spava::make_out(spava::kOutFinal));
       it.seg[0] = AttnSeg{0, r0 + rows, spava::kSegCausal, 0};
       v.push_back(it);
     }
@@ -348,10 +413,17 @@ spava_status launch_gather(const spava_plan* p, const void* k, const void* v, co
   return SPAVA_OK;
 }
 
+// Buffers only the two-stage flow uses (row partials and probe-score keys).
+struct TwoStageBufs {
+  float* row_o = nullptr;
+  float* row_lse = nullptr;
+  unsigned int* score_keys = nullptr;
+};
+
 template <int D>
 spava_status launch_attn(const spava_plan* p, const AttnItem* items, int n_items, const void* q, const void* k,
                          const void* v, const void* kp, const void* vp, void* o, float* lse, void* ws,
-                         cudaStream_t st) {
+                         cudaStream_t st, const TwoStageBufs& ts = TwoStageBufs()) {
   if (n_items == 0) return SPAVA_OK;
   CUtensorMap tmQ, tmK, tmV, tmKp, tmVp;
   spava_status s;
@@ -384,10 +456,18 @@ spava_status launch_attn(const spava_plan* p, const AttnItem* items, int n_items
   ap.err_word = err_word(p, ws);
   ap.wait_limit_ns = p->wait_limit_ns;
   ap.stall_producer = p->stall_producer;
+  ap.row_o = ts.row_o;
+  ap.row_lse = ts.row_lse;
+  ap.score_keys = ts.score_keys;
+  ap.n_visual = p->N;
+  ap.probe_r = p->R;
+  ap.scale = p->scale;
   using S = spava::AttnShape<D>;
   if ((s = ensure_smem(spava::attn_fwd_kernel<D>, S::kSmemBytes)) != SPAVA_OK) return s;
   const int grid = std::min(n_items, p->num_sms);
-  mark(p, items == p->d_items_dense ? kLabDense : kLabAttn, st);
+  mark(p, items == p->d_items_dense ? kLabDense
+             : items == p->d_items_local ? kLabAttnLocal
+             : items == p->d_items_remote ? kLabAttnRemote : kLabAttn, st);
   spava::attn_fwd_kernel<D><<<grid, S::kThreads, S::kSmemBytes, st>>>(tmQ, tmK, tmV, tmKp, tmVp, ap);
   SPAVA_CUDA(cudaGetLastError());
   ++g_last_launches;
@@ -510,6 +590,11 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   p->ws_lpart = o;
   o = align_up(o + static_cast<size_t>(n_hosts + 1) * hq * n_text * 4, 256);
   p->ws_total = o;
+  p->ws_row_o = o;
+  o = align_up(o + static_cast<size_t>(n_visual) * hq * head_dim * 4, 256);
+  p->ws_row_lse = o;
+  o = align_up(o + static_cast<size_t>(hq) * n_visual * 4, 256);
+  p->ws_total_two_stage = o;
 
   // device
   auto bail = [&](spava_status s) {
@@ -528,10 +613,14 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
 
   const auto pre = build_prefill_items(*p);
   const auto dense = build_dense_items(*p);
+  const auto local = build_local_items(*p);
+  const auto remote = build_remote_items(*p);
   const auto sc_pre = build_score_items(*p, n_hosts - 1);
   const auto sc_all = build_score_items(*p, n_hosts);
   p->n_items_pre = static_cast<int>(pre.size());
   p->n_items_dense = static_cast<int>(dense.size());
+  p->n_items_local = static_cast<int>(local.size());
+  p->n_items_remote = static_cast<int>(remote.size());
   p->n_score_pre = static_cast<int>(sc_pre.size());
   p->n_score_all = static_cast<int>(sc_all.size());
   const size_t b_off = align_up(off.size() * 4, 256);
@@ -539,7 +628,9 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   const size_t b_dense = align_up(dense.size() * sizeof(AttnItem), 256);
   const size_t b_spre = align_up(sc_pre.size() * sizeof(int4), 256);
   const size_t b_sall = align_up(sc_all.size() * sizeof(int4), 256);
-  std::vector<uint8_t> host(b_off + b_pre + b_dense + b_spre + b_sall, 0);
+  const size_t b_local = align_up(local.size() * sizeof(AttnItem), 256);
+  const size_t b_remote = align_up(remote.size() * sizeof(AttnItem), 256);
+  std::vector<uint8_t> host(b_off + b_pre + b_dense + b_spre + b_sall + b_local + b_remote, 0);
   size_t at = 0;
   std::memcpy(host.data() + at, off.data(), off.size() * 4);
   at += b_off;
@@ -550,6 +641,10 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   if (!sc_pre.empty()) std::memcpy(host.data() + at, sc_pre.data(), sc_pre.size() * sizeof(int4));
   at += b_spre;
   if (!sc_all.empty()) std::memcpy(host.data() + at, sc_all.data(), sc_all.size() * sizeof(int4));
+  at += b_sall;
+  if (!local.empty()) std::memcpy(host.data() + at, local.data(), local.size() * sizeof(AttnItem));
+  at += b_local;
+  if (!remote.empty()) std::memcpy(host.data() + at, remote.data(), remote.size() * sizeof(AttnItem));
   e = cudaMalloc(&p->dtab, host.size());
   if (e != cudaSuccess) return bail(fail(SPAVA_ERR_CUDA, "cudaMalloc(plan table): %s", cudaGetErrorString(e)));
   e = cudaMemcpy(p->dtab, host.data(), host.size(), cudaMemcpyHostToDevice);
@@ -560,6 +655,8 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   p->d_items_dense = reinterpret_cast<AttnItem*>(base + b_off + b_pre);
   p->d_score_pre = reinterpret_cast<int4*>(base + b_off + b_pre + b_dense);
   p->d_score_all = reinterpret_cast<int4*>(base + b_off + b_pre + b_dense + b_spre);
+  p->d_items_local = reinterpret_cast<AttnItem*>(base + b_off + b_pre + b_dense + b_spre + b_sall);
+  p->d_items_remote = reinterpret_cast<AttnItem*>(base + b_off + b_pre + b_dense + b_spre + b_sall + b_local);
   *out = p;
   return ok();
 }
@@ -705,6 +802,54 @@ spava_status spava_attn_prefill_noalloc(const spava_plan* p, const void* q, cons
   return spava_attn_prefill(p, q, k, v, o, lse, nullptr, nullptr, ws, stream);
 }
 
+size_t spava_two_stage_workspace_bytes(const spava_plan* p) { return p ? p->ws_total_two_stage : 0; }
+
+spava_status spava_attn_prefill_two_stage(const spava_plan* p, const void* q, const void* k, const void* v, void* o,
+                                          float* lse, float* scores_out, int32_t* idx_out, void* ws, void* stream) {
+  spava_status s;
+  if ((s = check_plan_ws(p, ws)) != SPAVA_OK) return s;
+  if (!q || !k || !v || !o || !lse) return fail(SPAVA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(SPAVA_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = begin_call(p, ws, st)) != SPAVA_OK) return s;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* scores = scores_out ? scores_out : reinterpret_cast<float*>(w + p->ws_scores);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + p->ws_idx);
+  void* kp = w + p->ws_kp;
+  void* vp = w + p->ws_vp;
+  TwoStageBufs ts;
+  ts.row_o = reinterpret_cast<float*>(w + p->ws_row_o);
+  ts.row_lse = reinterpret_cast<float*>(w + p->ws_row_lse);
+  ts.score_keys = reinterpret_cast<unsigned int*>(scores);  // keys, turned into scores in place
+  const size_t n_keys = static_cast<size_t>(p->hkv) * p->N;
+  const int grid_small = std::max(1, std::min(p->num_sms * 4, static_cast<int>((n_keys + 255) / 256)));
+  if (scores_needed(*p)) {
+    mark(p, kLabFill, st);
+    spava::fill_u32_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, n_keys, spava::kOrderedNegInf);
+    SPAVA_CUDA(cudaGetLastError());
+    ++g_last_launches;
+  }
+  // stage 1: local causal pass (+ fused probe scores, + text pieces)
+  s = p->d == 128 ? launch_attn<128>(p, p->d_items_local, p->n_items_local, q, k, v, nullptr, nullptr, o, lse, ws, st, ts)
+                  : launch_attn<64>(p, p->d_items_local, p->n_items_local, q, k, v, nullptr, nullptr, o, lse, ws, st, ts);
+  if (s != SPAVA_OK) return s;
+  if (scores_needed(*p)) {
+    mark(p, kLabFill, st);
+    spava::keys_to_scores_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, n_keys);
+    SPAVA_CUDA(cudaGetLastError());
+    ++g_last_launches;
+    if ((s = launch_select(p, scores, idx, st, k, v, kp, vp)) != SPAVA_OK) return s;
+  }
+  // stage 2: remote pass over [anchor | passing], lse-merged with the local partials
+  s = p->d == 128 ? launch_attn<128>(p, p->d_items_remote, p->n_items_remote, q, k, v, kp, vp, o, lse, ws, st, ts)
+                  : launch_attn<64>(p, p->d_items_remote, p->n_items_remote, q, k, v, kp, vp, o, lse, ws, st, ts);
+  if (s != SPAVA_OK) return s;
+  if ((s = launch_merge(p, o, lse, ws, st)) != SPAVA_OK) return s;
+  mark(p, -1, st);
+  return ok();
+}
+
 spava_status spava_dense_causal(const spava_plan* p, const void* q, const void* k, const void* v, void* o, float* lse,
                                 void* ws, void* stream) {
   spava_status s;
@@ -769,6 +914,9 @@ const char* spava_kernel_name(int32_t label) {
     case kLabMerge: return "lse_merge";
     case kLabDense: return "attention_dense";
     case kLabSelectGather: return "select_gather";
+    case kLabFill: return "score_keys";
+    case kLabAttnLocal: return "attention_local";
+    case kLabAttnRemote: return "attention_remote";
   }
   return "unknown";
 }

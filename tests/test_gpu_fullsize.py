@@ -155,3 +155,41 @@ def test_fullsize_dense_causal_256k(fullsize_run):
     do = np.abs(o[rt, ht].float().cpu().numpy() - O_ref).max()
     dl = np.abs(lse[ht, rt].cpu().numpy() - L_ref).max()
     assert do <= O_TOL and dl <= LSE_TOL, (do, dl)
+
+
+def test_fullsize_two_stage_flow(fullsize_run):
+    """The two-stage flow (local pass with fused probe scores, remote pass merged
+    through the lse) on the same full-size inputs: fused scores within tolerance of the
+    oracle, selection bit-exact on its own scores, sampled outputs against the oracle
+    re-run with its indices."""
+    r = fullsize_run
+    cfg = r["cfg"]
+    if cfg.name not in ("128k", "stress"):
+        pytest.skip("two-stage flow checked at full size on the 128k and stress workloads")
+    dev, plan = r["dev"], r["plan"]
+    ws = plan.new_workspace(two_stage=True)
+    scores = torch.empty((cfg.hkv, cfg.n_visual), dtype=torch.float32, device="cuda")
+    idx = torch.empty(plan.idx_shape(), dtype=torch.int32, device="cuda")
+    o, lse = sab.attn_prefill_two_stage(plan, dev["q"], dev["k"], dev["v"], scores_out=scores, idx_out=idx,
+                                        workspace=ws)
+    sab.check_device_error(plan, ws)
+    off = orc.host_offsets(r["sizes"])
+    q, k, v = (LazyF64(r["g"][x]) for x in ("q", "k", "v"))
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    sc = scores.cpu().numpy()
+    hosts = range(cfg.n_hosts - 1)
+    ref, tol = _score_tolerance_and_ref(q, k, off, cfg.probe_r, scale, hosts)
+    for (h, g), val in ref.items():
+        a, e = int(off[h]), int(off[h + 1])
+        assert (np.abs(sc[g, a:e] - val) <= tol[(h, g)]).all(), (cfg.name, h, g)
+    sel = idx.cpu().numpy().astype(np.int64)
+    np.testing.assert_array_equal(sel, orc.select_passing(sc, off, cfg.anchor, cfg.passing))
+    rng = np.random.default_rng(cfg.seed + 1)
+    rows, heads = _sample_rows(cfg, off, rng)
+    O_ref, L_ref = orc.attention_rows(q, k, v, off, cfg.anchor, sel, scale, rows, heads)
+    rt, ht = torch.tensor(rows, device="cuda"), torch.tensor(heads, device="cuda")
+    do = np.abs(o[rt, ht].float().cpu().numpy() - O_ref).max()
+    dl = np.abs(lse[ht, rt].cpu().numpy() - L_ref).max()
+    assert do <= O_TOL and dl <= LSE_TOL, (cfg.name, do, dl)
+    del ws
+    torch.cuda.empty_cache()

@@ -225,3 +225,40 @@ def test_bad_arguments_raise_before_launch():
                                 ctypes.c_void_p(ws.data_ptr()), None, None, ctypes.c_void_p(ws.data_ptr()), None)
     assert st == 1  # misaligned q
     plan.close()
+
+
+# ---------------------------------------------------------------- two-stage flow
+@pytest.mark.parametrize("name", list(CASES))
+def test_two_stage_prefill_matches_oracle(name):
+    """Local pass with fused probe scores -> select/gather -> remote pass merged through
+    the lse: scores within tolerance of the oracle, selection bit-exact on its own fp32
+    scores, O/lse against the oracle re-run with its indices."""
+    cfg, sizes = CASES[name]
+    cfg = cfg.with_(uneven=None)
+    g, f64, dev = inputs(cfg)
+    sizes = _sizes(cfg, sizes)
+    plan = make_plan(sab, cfg, sizes)
+    off = orc.host_offsets(sizes)
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    ws = plan.new_workspace(two_stage=True)
+    scores = torch.full((cfg.hkv, cfg.n_visual), float("nan"), device="cuda")
+    idx = torch.full(plan.idx_shape(), -1, dtype=torch.int32, device="cuda")
+    o, lse = sab.attn_prefill_two_stage(plan, dev["q"], dev["k"], dev["v"], scores_out=scores, idx_out=idx,
+                                        workspace=ws)
+    sab.check_device_error(plan, ws)
+    torch.cuda.synchronize()
+    H = cfg.n_hosts
+    sel = idx.cpu().numpy().astype(np.int64)
+    if H > 1 and cfg.passing > 0:
+        sc = scores.cpu().numpy()
+        n_sc = int(off[H - 1])
+        ref_scores = orc.probe_scores(f64["q"], f64["k"], off, cfg.probe_r, scale)
+        tol = score_tolerance(f64["q"], f64["k"], off, cfg.probe_r, scale)
+        err = np.abs(sc[:, :n_sc] - ref_scores[:, :n_sc])
+        assert (err <= tol[:, :n_sc]).all(), f"fused score error {np.nanmax(err)}"
+        np.testing.assert_array_equal(sel, orc.select_passing(sc, off, cfg.anchor, cfg.passing))
+        check_selection_vs_fp64(sel, ref_scores, off, cfg.anchor, cfg.passing)
+    O_ref, L_ref = orc.approx_attention(f64["q"], f64["k"], f64["v"], off, cfg.anchor,
+                                        sel if H > 1 else None, scale)
+    compare_attention(o, lse, O_ref, L_ref, "two-stage " + name)
+    plan.close()
