@@ -47,6 +47,8 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
 // them from global memory on every pass (any segment length).
 // With kGather the CTA then copies its P passing rows of K and V into
 // k_pass/v_pass[g][h] (16 bytes per thread), so the prefill needs no separate gather.
+constexpr int kGatherUnroll = 4;
+
 struct GatherArgs {
   const uint4* k;
   const uint4* v;
@@ -158,14 +160,32 @@ __global__ void __launch_bounds__(1024) select_topp_kernel(const float* __restri
   }
   if (kGather) {
     __syncthreads();  // the block's index writes are visible to the block after this
-    const int cpr = ga.chunks_per_row;
+    // kGatherUnroll rows' chunks per thread are loaded before any is stored, so each
+    // SM keeps kGatherUnroll * 2 * 16 B * blockDim.x of K/V reads in flight.
+    const int cpr = ga.chunks_per_row;  // a power of two (8 or 16)
+    const int cpr_shift = __ffs(cpr) - 1;
+    const int total = passing * cpr;
     const size_t dst0 = ((static_cast<size_t>(g) * ga.hosts_m1 + h) * passing) * cpr;
-    for (int t = tid; t < passing * cpr; t += nt) {
-      const int r = t / cpr, ch = t - r * cpr;
-      const int tok = out[r];
-      const size_t src = (static_cast<size_t>(tok) * hkv + g) * cpr + ch;
-      ga.kp[dst0 + t] = __ldg(ga.k + src);
-      ga.vp[dst0 + t] = __ldg(ga.v + src);
+    for (int t0 = tid; t0 < total; t0 += kGatherUnroll * nt) {
+      uint4 kv[kGatherUnroll], vv[kGatherUnroll];
+#pragma unroll
+      for (int u = 0; u < kGatherUnroll; ++u) {
+        const int t = t0 + u * nt;
+        if (t < total) {
+          const int r = t >> cpr_shift, ch = t & (cpr - 1);
+          const size_t src = (static_cast<size_t>(out[r]) * hkv + g) * cpr + ch;
+          kv[u] = __ldg(ga.k + src);
+          vv[u] = __ldg(ga.v + src);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kGatherUnroll; ++u) {
+        const int t = t0 + u * nt;
+        if (t < total) {
+          ga.kp[dst0 + t] = kv[u];
+          ga.vp[dst0 + t] = vv[u];
+        }
+      }
     }
   }
 }

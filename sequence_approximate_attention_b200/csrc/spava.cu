@@ -623,40 +623,33 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   p->n_items_remote = static_cast<int>(remote.size());
   p->n_score_pre = static_cast<int>(sc_pre.size());
   p->n_score_all = static_cast<int>(sc_all.size());
-  const size_t b_off = align_up(off.size() * 4, 256);
-  const size_t b_pre = align_up(pre.size() * sizeof(AttnItem), 256);
-  const size_t b_dense = align_up(dense.size() * sizeof(AttnItem), 256);
-  const size_t b_spre = align_up(sc_pre.size() * sizeof(int4), 256);
-  const size_t b_sall = align_up(sc_all.size() * sizeof(int4), 256);
-  const size_t b_local = align_up(local.size() * sizeof(AttnItem), 256);
-  const size_t b_remote = align_up(remote.size() * sizeof(AttnItem), 256);
-  std::vector<uint8_t> host(b_off + b_pre + b_dense + b_spre + b_sall + b_local + b_remote, 0);
-  size_t at = 0;
-  std::memcpy(host.data() + at, off.data(), off.size() * 4);
-  at += b_off;
-  if (!pre.empty()) std::memcpy(host.data() + at, pre.data(), pre.size() * sizeof(AttnItem));
-  at += b_pre;
-  if (!dense.empty()) std::memcpy(host.data() + at, dense.data(), dense.size() * sizeof(AttnItem));
-  at += b_dense;
-  if (!sc_pre.empty()) std::memcpy(host.data() + at, sc_pre.data(), sc_pre.size() * sizeof(int4));
-  at += b_spre;
-  if (!sc_all.empty()) std::memcpy(host.data() + at, sc_all.data(), sc_all.size() * sizeof(int4));
-  at += b_sall;
-  if (!local.empty()) std::memcpy(host.data() + at, local.data(), local.size() * sizeof(AttnItem));
-  at += b_local;
-  if (!remote.empty()) std::memcpy(host.data() + at, remote.data(), remote.size() * sizeof(AttnItem));
+  // One device table, each array 256-byte aligned.
+  std::vector<uint8_t> host;
+  auto put = [&host](const void* src, size_t bytes) {
+    const size_t at = host.size();
+    host.resize(align_up(at + bytes, 256), 0);
+    if (bytes) std::memcpy(host.data() + at, src, bytes);
+    return at;
+  };
+  const size_t o_off = put(off.data(), off.size() * 4);
+  const size_t o_pre = put(pre.data(), pre.size() * sizeof(AttnItem));
+  const size_t o_dense = put(dense.data(), dense.size() * sizeof(AttnItem));
+  const size_t o_spre = put(sc_pre.data(), sc_pre.size() * sizeof(int4));
+  const size_t o_sall = put(sc_all.data(), sc_all.size() * sizeof(int4));
+  const size_t o_local = put(local.data(), local.size() * sizeof(AttnItem));
+  const size_t o_remote = put(remote.data(), remote.size() * sizeof(AttnItem));
   e = cudaMalloc(&p->dtab, host.size());
   if (e != cudaSuccess) return bail(fail(SPAVA_ERR_CUDA, "cudaMalloc(plan table): %s", cudaGetErrorString(e)));
   e = cudaMemcpy(p->dtab, host.data(), host.size(), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return bail(fail(SPAVA_ERR_CUDA, "cudaMemcpy(plan table): %s", cudaGetErrorString(e)));
   uint8_t* base = static_cast<uint8_t*>(p->dtab);
-  p->d_off = reinterpret_cast<int*>(base);
-  p->d_items_pre = reinterpret_cast<AttnItem*>(base + b_off);
-  p->d_items_dense = reinterpret_cast<AttnItem*>(base + b_off + b_pre);
-  p->d_score_pre = reinterpret_cast<int4*>(base + b_off + b_pre + b_dense);
-  p->d_score_all = reinterpret_cast<int4*>(base + b_off + b_pre + b_dense + b_spre);
-  p->d_items_local = reinterpret_cast<AttnItem*>(base + b_off + b_pre + b_dense + b_spre + b_sall);
-  p->d_items_remote = reinterpret_cast<AttnItem*>(base + b_off + b_pre + b_dense + b_spre + b_sall + b_local);
+  p->d_off = reinterpret_cast<int*>(base + o_off);
+  p->d_items_pre = reinterpret_cast<AttnItem*>(base + o_pre);
+  p->d_items_dense = reinterpret_cast<AttnItem*>(base + o_dense);
+  p->d_score_pre = reinterpret_cast<int4*>(base + o_spre);
+  p->d_score_all = reinterpret_cast<int4*>(base + o_sall);
+  p->d_items_local = reinterpret_cast<AttnItem*>(base + o_local);
+  p->d_items_remote = reinterpret_cast<AttnItem*>(base + o_remote);
   *out = p;
   return ok();
 }
