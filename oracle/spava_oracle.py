@@ -27,7 +27,10 @@ Readings taken where they are silent (each is a parameter of this oracle):
   R1  score of key j of host h, KV head g: the max, over the last R query rows i
       of host h with i >= j and over the query heads c of group g, of
       s_c(i, j) = (q_{i,c} . k_{j,g}) * scale, scale = d^-1/2.  (max over heads:
-      parity unpinned -- no page value fixes sum vs max.)
+      parity unpinned -- no page value fixes sum vs max.)  Switchable
+      (``head_reduce``): with "sum" or "mean" each head first takes its own max
+      over the probe rows, m_c(j), and the group's score is sum_c m_c(j) or its
+      mean; "max" is max_c m_c(j), the default above.
   R2  causal inside the probe: probe row i never scores a key j > i.
   R3  host 0's anchor positions [0, A) are not passing candidates, so no key is
       attended twice by a later host (parity unpinned -- a plan-level reading).
@@ -73,12 +76,18 @@ def _groups(hq: int, hkv: int) -> int:
     return hq // hkv
 
 
+HEAD_REDUCE = ("max", "sum", "mean")
+
+
 def probe_scores(q: np.ndarray, k: np.ndarray, off: np.ndarray, probe_r: int,
-                 scale: float) -> np.ndarray:
+                 scale: float, head_reduce: str = "max") -> np.ndarray:
     """Query-to-context scores of every visual key (readings R1, R2).
 
     q [tokens, hq, d], k [tokens, hkv, d] float64; returns float64 [hkv, N].
+    ``head_reduce`` combines the per-head probe maxima of a KV group (R1).
     """
+    if head_reduce not in HEAD_REDUCE:
+        raise ValueError(f"head_reduce must be one of {HEAD_REDUCE}")
     hq, hkv = q.shape[1], k.shape[1]
     G = _groups(hq, hkv)
     H = len(off) - 1
@@ -95,7 +104,13 @@ def probe_scores(q: np.ndarray, k: np.ndarray, off: np.ndarray, probe_r: int,
             qg = q[e - probe_r:e, g * G:(g + 1) * G, :]              # [R, G, d]
             s = np.matmul(qg.transpose(1, 0, 2), k[a:e, g, :].T)     # [G, R, B]
             s = np.where(visible[None], s * scale, -np.inf)
-            scores[g, a:e] = s.max(axis=(0, 1))
+            per_head = s.max(axis=1)                                 # [G, B]: m_c(j)
+            if head_reduce == "max":
+                scores[g, a:e] = per_head.max(axis=0)
+            elif head_reduce == "sum":
+                scores[g, a:e] = per_head.sum(axis=0)
+            else:
+                scores[g, a:e] = per_head.sum(axis=0) / G
     return scores
 
 
@@ -251,7 +266,7 @@ def lse_merge(o1: np.ndarray, l1: np.ndarray, o2: np.ndarray, l2: np.ndarray):
 
 def prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, host_sizes: Sequence[int],
             anchor: int, passing: int, probe_r: int, scale: Optional[float] = None,
-            sel: Optional[np.ndarray] = None, rows=None) -> Dict[str, np.ndarray]:
+            sel: Optional[np.ndarray] = None, rows=None, head_reduce: str = "max") -> Dict[str, np.ndarray]:
     """Whole prefill: split -> score -> select -> approximate attention.
 
     q/k/v are float64 (see ``bf16_bits_to_f64``).  If ``sel`` is given it replaces
@@ -263,7 +278,7 @@ def prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, host_sizes: Sequence[in
         scale = 1.0 / np.sqrt(d)
     off = host_offsets(host_sizes)
     out: Dict[str, np.ndarray] = {"offsets": off}
-    out["scores"] = probe_scores(q, k, off, probe_r, scale)
+    out["scores"] = probe_scores(q, k, off, probe_r, scale, head_reduce)
     out["sel"] = select_passing(out["scores"], off, anchor, passing) if sel is None else sel
     if rows is None:
         out["O"], out["lse"] = approx_attention(q, k, v, off, anchor, out["sel"], scale)

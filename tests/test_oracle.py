@@ -233,6 +233,58 @@ def test_scores_brute_force():
                     assert got[g, j] >= q[e - 1, c] @ k[j, g] * scale - 1e-12
 
 
+@pytest.mark.parametrize("mode", ["sum", "mean"])
+def test_scores_head_reduce_brute_force(mode):
+    """Switchable reading R1: per-head max over the probe rows, then sum or mean over
+    the group's heads -- a pure-Python triple loop on tiny inputs."""
+    rng = np.random.default_rng(5)
+    sizes = [11, 14, 9]
+    hq, hkv, d, R = 6, 2, 4, 5
+    q, k, _ = _rand_qkv(rng, sum(sizes), hq, hkv, d)
+    scale = 0.6
+    off = orc.host_offsets(sizes)
+    got = orc.probe_scores(q, k, off, R, scale, head_reduce=mode)
+    G = hq // hkv
+    for h in range(len(sizes)):
+        a, e = int(off[h]), int(off[h + 1])
+        for g in range(hkv):
+            for j in range(a, e):
+                total = 0.0
+                for c in range(g * G, (g + 1) * G):
+                    best = -math.inf
+                    for i in range(max(j, e - R), e):
+                        best = max(best, sum(q[i, c, t] * k[j, g, t] for t in range(d)) * scale)
+                    total += best
+                want = total if mode == "sum" else total / G
+                assert got[g, j] == pytest.approx(want, rel=1e-13, abs=1e-13)
+
+
+def test_scores_head_reduce_decomposes_over_heads():
+    """sum over heads = the sum of max-mode scores of the one-head-per-group problems
+    (query head t of every group alone); the modes agree when a group has one head;
+    mean = sum / G."""
+    cfg = CONFIGS["tiny"].with_(hq=6, hkv=2, head_dim=16, n_visual=192, n_hosts=3, anchor=16, passing=8,
+                                probe_r=8)
+    g = generate(cfg)
+    q, k = orc.bf16_bits_to_f64(g["q"]), orc.bf16_bits_to_f64(g["k"])
+    off = orc.host_offsets(g["host_sizes"])
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    G = cfg.hq // cfg.hkv
+    s_sum = orc.probe_scores(q, k, off, cfg.probe_r, scale, "sum")
+    parts = [orc.probe_scores(q[:, [gg * G + t for gg in range(cfg.hkv)]],
+                              k, off, cfg.probe_r, scale, "max") for t in range(G)]
+    np.testing.assert_allclose(s_sum, sum(parts), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(orc.probe_scores(q, k, off, cfg.probe_r, scale, "mean"), s_sum / G,
+                               rtol=1e-14, atol=1e-14)
+    one = [gg * G for gg in range(cfg.hkv)]
+    q1 = q[:, one]
+    ref = orc.probe_scores(q1, k, off, cfg.probe_r, scale, "max")
+    for mode in ("sum", "mean"):
+        np.testing.assert_array_equal(orc.probe_scores(q1, k, off, cfg.probe_r, scale, mode), ref)
+    with pytest.raises(ValueError):
+        orc.probe_scores(q, k, off, cfg.probe_r, scale, "median")
+
+
 def _brute_select(vals, lo, P):
     order = sorted(range(len(vals)), key=lambda t: (-float(vals[t]), t))
     return sorted(lo + t for t in order[:P])
