@@ -96,6 +96,22 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
 /* Free a plan and its device table (synchronises the device first).  NULL is OK. */
 spava_status spava_plan_destroy(spava_plan* plan);
 
+/* How the query heads of a KV group combine into one score per key.  The pages say
+ * only that hosts pick their passing keys by query-to-context attention scores (APB-V
+ * technical summary, 1. Framework design, "Approximate attention mechanism"); with
+ * m_c(j) = max over the probe rows i >= j of q_{i,c} . k_j (query head c):
+ *   SPAVA_SCORE_MAX   score(g, j) = scale * max_c m_c(j)          (default)
+ *   SPAVA_SCORE_SUM   score(g, j) = scale * sum_c m_c(j)
+ *   SPAVA_SCORE_MEAN  score(g, j) = scale * sum_c m_c(j) / G
+ * over the G query heads c of KV head g. */
+typedef enum { SPAVA_SCORE_MAX = 0, SPAVA_SCORE_SUM = 1, SPAVA_SCORE_MEAN = 2 } spava_score_reduce;
+
+/* Select the head reduction (spava_score_reduce) for this plan's later calls
+ * (spava_score_select, spava_attn_prefill and its variants).  Host-side only; the
+ * workspace sizes do not depend on it.  Returns SPAVA_ERR_INVALID_ARG for a NULL plan
+ * or an unknown mode. */
+spava_status spava_plan_set_score_reduce(spava_plan* plan, int32_t mode);
+
 /* Bytes of scratch the calls below need (scores, indices, passing K/V, text
  * partials, scheduler counters, error word).  0 if plan is NULL. */
 size_t spava_workspace_bytes(const spava_plan* plan);

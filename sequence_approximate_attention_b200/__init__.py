@@ -86,6 +86,16 @@ class Plan:
         n = self.two_stage_workspace_bytes if two_stage else self.workspace_bytes
         return torch.zeros(max(n, 256), dtype=torch.uint8, device=self.device)
 
+    SCORE_REDUCE = {"max": 0, "sum": 1, "mean": 2}
+
+    def set_score_reduce(self, mode: str) -> None:
+        """spava_plan_set_score_reduce: how the query heads of a KV group combine the
+        probe scores ("max" default, "sum", "mean" of the per-head maxima)."""
+        if mode not in self.SCORE_REDUCE:
+            raise ValueError(f"score reduction must be one of {sorted(self.SCORE_REDUCE)}")
+        _lib.check(self.lib.spava_plan_set_score_reduce(self._h, self.SCORE_REDUCE[mode]), "spava_plan_set_score_reduce")
+        self.score_reduce = mode
+
     def set_debug(self, wait_limit_ns: int = 0, stall_producer: bool = False) -> None:
         _lib.check(self.lib.spava_plan_set_debug(self._h, int(wait_limit_ns), int(bool(stall_producer))),
                    "spava_plan_set_debug")

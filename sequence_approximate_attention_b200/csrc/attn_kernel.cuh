@@ -82,7 +82,9 @@ struct AttnParams {
   // two-stage flow
   float* row_o;               // [N][hq][D] fp32 partials of visual rows
   float* row_lse;             // [hq][N]
-  unsigned int* score_keys;   // [hkv][N] ordered probe-score keys, max-reduced
+  unsigned int* score_keys;   // ordered probe-score keys, max-reduced: [hkv][N], or
+                              // [hq][N] (one row per query head) when score_per_qhead
+  int score_per_qhead;        // the heads are combined later (sum / mean reductions)
   int n_visual;
   int probe_r;
   float scale;                // softmax scale (scores are max(q.k) * scale)
@@ -516,7 +518,9 @@ __global__ void __launch_bounds__(384, 1)
           // (P has not been stored yet) and is re-read 32 columns at a time.
           const bool probe_row = qpos >= sg.aux - p.probe_r && qpos < sg.aux && (i * 128 + row) < it.q_rows;
           if (__any_sync(FULL, probe_row)) {
-            unsigned int* keys = p.score_keys + static_cast<size_t>(it.q_head / p.group) * p.n_visual + kpos0;
+            unsigned int* keys =
+                p.score_keys + static_cast<size_t>(p.score_per_qhead ? it.q_head : it.q_head / p.group) * p.n_visual +
+                kpos0;
             int lim = valid;
             if (causal) lim = min(lim, qpos - kpos0 + 1);
 #pragma unroll 1

@@ -2,15 +2,18 @@
 // 1. Framework design, "Approximate attention mechanism": every host ranks its
 // local keys by query-to-context attention scores).
 //
-//   score(g, j) = scale * max over probe rows i in [e-R, e), i >= j, and query heads
-//                 c of group g of (q_{i,c} . k_{j,g}),   e = end of j's host block.
+//   m_c(j)   = max over probe rows i in [e-R, e), i >= j, of (q_{i,c} . k_{j,g})
+//   score(g, j) = scale * reduce over the query heads c of group g of m_c(j),
+//   e = end of j's host block; reduce = max (default), sum or mean (the pages leave
+//   the combination open; max over heads and rows is the plainest reading).
 //
 // The product is computed transposed, S^T = K_tile * Qprobe^T, so that each TMEM
 // lane holds one key and the max over (probe row, head) is a per-thread reduction
 // along the lane's columns (no cross-thread reduction).  The probe queries of one
-// (host, KV group) form the MMA's N dimension: rows ordered (token, head) exactly as
-// a TMA box (64 x G x Rc) of q lands in shared memory, cut into chunks of at most
-// 256 columns.  Work item = one 128-key tile of one (host, KV head).
+// (host, KV group) form the MMA's N dimension, ordered (head, token): one TMA box
+// (64 x 1 x Rc) per query head, so head c owns columns [c Rc, c Rc + Rc) of a chunk
+// of Rc probe tokens (Rc G <= 256).  Work item = one 128-key tile of one (host, KV
+// head).
 //
 // CTA = 256 threads: warp 0 TMA, warp 1 MMA, warp 2 TMEM allocator,
 // warps 4-7 epilogue (lane = key).  TMEM holds two 256-column accumulators so the
@@ -28,6 +31,7 @@ struct ScoreParams {
   int group;         // G = hq / hkv
   int chunk_tokens;  // Rc probe tokens per N chunk (Rc * G <= 256, multiple of 16)
   int n_chunks;      // ceil(R / Rc)
+  int head_reduce;   // 0 max, 1 sum, 2 mean over the group's query heads
   int n_visual;      // N (row stride of scores)
   float scale;
   float* scores;     // [hkv][N]
@@ -50,6 +54,7 @@ struct ScoreShape {
   static constexpr int kItemBytes = kMaxLocalItems * 16;
   static constexpr int kSmemMax = 232448;  // opt-in limit per CTA on sm_100
   static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kMaxGroup = 16;  // query heads per KV head
   // Bytes of dynamic shared memory for a given pipeline (plus alignment slack).
   static constexpr int smem_bytes(int q_bufs, int q_buf_bytes, int k_stages) {
     return q_bufs * q_buf_bytes + k_stages * kKTileBytes + kBarBytes + kItemBytes + 1024;
@@ -170,8 +175,9 @@ __global__ void __launch_bounds__(256, 1)
         if (lane == 0) {
           mbar_arrive_expect_tx(q_full + b, static_cast<uint32_t>(S::kHalves * p.chunk_tokens * G * 128));
           for (int hh = 0; hh < S::kHalves; ++hh)
-            tma_load_3d(sQ + b * p.q_buf_bytes + hh * (p.chunk_tokens * G * 128), &tmQp, q_full + b, hh * 64,
-                        it.y * G, it.w - p.probe_r + c * p.chunk_tokens);
+            for (int h = 0; h < G; ++h)
+              tma_load_3d(sQ + b * p.q_buf_bytes + hh * (p.chunk_tokens * G * 128) + h * (p.chunk_tokens * 128), &tmQp,
+                          q_full + b, hh * 64, it.y * G + h, it.w - p.probe_r + c * p.chunk_tokens);
         }
         __syncwarp();
         ++qloads[b];
@@ -211,8 +217,9 @@ __global__ void __launch_bounds__(256, 1)
           if (!ok) break;
         }
         tc_fence_after();
-        const int rc = min(p.chunk_tokens, p.probe_r - c * p.chunk_tokens);
-        const int nc = rc * G;
+        // All Rc G columns: with (head, token) order a short last chunk's probe rows
+        // are not a prefix; the epilogue masks the rest.
+        const int nc = p.chunk_tokens * G;
         if (lane == 0) {
           const uint32_t idesc = idesc_bf16_f32(128, nc, 0, 0);
           const uint32_t ka = smem_u32(sK + slot * S::kKTileBytes);
@@ -252,55 +259,85 @@ __global__ void __launch_bounds__(256, 1)
     const int qd = warp & 3;
     const int row = qd * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    const int Rc = p.chunk_tokens;
     bool ok = true;
     for (int li = 0; li < n_local && ok; ++li) {
       const int4 it = s_items[li];
       const int j = it.z + row;  // key position
       const int e = it.w;
-      float mx = -INFINITY;
+      const bool by_head = p.head_reduce != 0;
+      float mx_all = -INFINITY;   // max over heads and rows
+      float mh[S::kMaxGroup];     // sum / mean: m_c(j) of each query head (indexed at run time)
+      if (by_head) {
+#pragma unroll 1
+        for (int h = 0; h < G; ++h) mh[h] = -INFINITY;
+      }
       for (int c = 0; c < p.n_chunks; ++c) {
         const int u = li * p.n_chunks + c, b = u & 1;
         ok = __all_sync(FULL, mbar_wait(acc_full + b, (u >> 1) & 1, wc, kErrWaitMma));
         if (!ok) break;
         tc_fence_after();
-        const int rc = min(p.chunk_tokens, p.probe_r - c * p.chunk_tokens);
-        const int nc = rc * G;
-        // Column n is probe token c*Rc + n/G, i.e. row e - R + c*Rc + n/G; it may score
-        // key j iff that row >= j, i.e. n >= G * (j - (e - R + c*Rc)).
-        const int col_min = G * (j - (e - p.probe_r + c * p.chunk_tokens));
-        int n0 = 0;
-        // Whole 128-column blocks: one TMEM load each, then a three-input max tree.
-        for (; n0 + 128 <= nc; n0 += 128) {
-          uint32_t v[128];
-          tmem_ld_x128(tl + b * 256 + n0, v);
-          if (col_min > n0) {
+        const int row0 = e - p.probe_r + c * Rc;         // first probe row of the chunk
+        const int rc = min(Rc, p.probe_r - c * Rc);      // probe rows in it (a multiple of 16)
+        const uint32_t ta = tl + b * 256;
+        if (!by_head && rc == Rc && it.z + 127 < row0) {
+          // Max over heads and rows with every column visible to every key of the
+          // tile: order-free, whole 128-column TMEM loads and a three-input max tree.
+          const int nc = Rc * G;
+          int n0 = 0;
+#pragma unroll 1  // one 128-register block live at a time
+          for (; n0 + 128 <= nc; n0 += 128) {
+            uint32_t v[128];
+            tmem_ld_x128(ta + n0, v);
+            float m8[8];
 #pragma unroll
-            for (int t = 0; t < 128; ++t)
-              if (n0 + t < col_min) v[t] = 0xff800000u;  // -inf: probe row before key j
+            for (int k = 0; k < 8; ++k) m8[k] = fmaxf(__uint_as_float(v[k]), __uint_as_float(v[k + 8]));
+#pragma unroll
+            for (int t = 16; t < 128; t += 16)
+#pragma unroll
+              for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], __uint_as_float(v[t + k]), __uint_as_float(v[t + 8 + k]));
+            mx_all = fmax3(mx_all, fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])),
+                           -INFINITY);
           }
-          float m8[8];
+          for (; n0 < nc; n0 += 16) {
+            uint32_t v[16];
+            tmem_ld_x16(ta + n0, v);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) m8[k] = fmaxf(__uint_as_float(v[k]), __uint_as_float(v[k + 8]));
+            for (int t = 0; t < 16; ++t) mx_all = fmaxf(mx_all, __uint_as_float(v[t]));
+          }
+        } else {
+          // Per head h: columns [h Rc, h Rc + rc); probe row row0 + t scores key j iff
+          // row0 + t >= j.
+          const int t_min = j - row0;
+#pragma unroll 1
+          for (int h = 0; h < G; ++h) {
+            float m = -INFINITY;
+            for (int t0 = 0; t0 < rc; t0 += 16) {
+              uint32_t v[16];
+              tmem_ld_x16(ta + h * Rc + t0, v);
 #pragma unroll
-          for (int t = 16; t < 128; t += 16)
-#pragma unroll
-            for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], __uint_as_float(v[t + k]), __uint_as_float(v[t + 8 + k]));
-          mx = fmax3(mx, fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])), -INFINITY);
-        }
-        // Remaining columns (chunks that are not a multiple of 128) in 16-column loads.
-        for (; n0 < nc; n0 += 16) {
-          uint32_t v[16];
-          tmem_ld_x16(tl + b * 256 + n0, v);
-#pragma unroll
-          for (int t = 0; t < 16; ++t)
-            if (n0 + t >= col_min) mx = fmaxf(mx, __uint_as_float(v[t]));
+              for (int t = 0; t < 16; ++t)
+                if (t0 + t >= t_min) m = fmaxf(m, __uint_as_float(v[t]));
+            }
+            if (by_head)
+              mh[h] = fmaxf(mh[h], m);
+            else
+              mx_all = fmaxf(mx_all, m);
+          }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty + b);
       }
       if (!ok) break;
-      if (j < e) p.scores[static_cast<size_t>(it.y) * p.n_visual + j] = mx * p.scale;
+      float r = mx_all;
+      if (by_head) {
+        r = 0.f;
+#pragma unroll 1
+        for (int h = 0; h < G; ++h) r += mh[h];
+        if (p.head_reduce == 2) r = r / static_cast<float>(G);
+      }
+      if (j < e) p.scores[static_cast<size_t>(it.y) * p.n_visual + j] = r * p.scale;
     }
   }
 

@@ -203,6 +203,22 @@ __global__ void __launch_bounds__(256) keys_to_scores_kernel(uint32_t* __restric
     p[t] = __float_as_uint(key_to_float(p[t]));
 }
 
+// Two-stage flow with a sum or mean head reduction: keys hold each query head's max
+// over its probe rows, [hq][N]; scores[g][j] = sum (or mean) over the G heads of
+// group g.  mode 1 sum, 2 mean.
+__global__ void __launch_bounds__(256) combine_head_keys_kernel(const uint32_t* __restrict__ keys,
+                                                                 float* __restrict__ scores, int hkv, int group,
+                                                                 size_t n, int mode) {
+  const size_t total = static_cast<size_t>(hkv) * n;
+  for (size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t g = t / n, j = t - g * n;
+    float r = 0.f;
+    for (int c = 0; c < group; ++c) r += key_to_float(__ldg(keys + (g * group + c) * n + j));
+    scores[t] = mode == 2 ? r / static_cast<float>(group) : r;
+  }
+}
+
 // k_pass[g][h][j][:] = k[idx[h][g][j]][g][:] (same for v), 16 bytes per thread.
 __global__ void __launch_bounds__(256) gather_passing_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                                               const int32_t* __restrict__ idx, uint4* __restrict__ kp,

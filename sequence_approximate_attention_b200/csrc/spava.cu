@@ -101,6 +101,7 @@ struct spava_plan {
   int device = 0, num_sms = 0;
   // score chunking: Rc probe tokens per MMA N chunk
   int rc = 0, n_chunks = 0;
+  int score_reduce = SPAVA_SCORE_MAX;  // spava_plan_set_score_reduce
   // device table (owned)
   void* dtab = nullptr;
   int* d_off = nullptr;
@@ -118,7 +119,7 @@ struct spava_plan {
   int n_score_all = 0;
   // workspace layout
   size_t ws_err = 0, ws_scores = 0, ws_idx = 0, ws_kp = 0, ws_vp = 0, ws_opart = 0, ws_lpart = 0, ws_total = 0;
-  size_t ws_row_o = 0, ws_row_lse = 0, ws_total_two_stage = 0;  // two-stage flow only
+  size_t ws_row_o = 0, ws_row_lse = 0, ws_qkeys = 0, ws_total_two_stage = 0;  // two-stage flow only
   // debug knobs
   uint64_t wait_limit_ns = spava::kDefaultWaitLimitNs;
   int stall_producer = 0;
@@ -337,7 +338,7 @@ spava_status launch_score(const spava_plan* p, const void* q, const void* k, flo
   spava_status s;
   if ((s = make_map(&tmK, k, D, p->hkv, p->N + p->T, 1, 128)) != SPAVA_OK) return s;
   const int G = p->hq / p->hkv;
-  if ((s = make_map(&tmQp, q, D, p->hq, p->N + p->T, G, p->rc)) != SPAVA_OK) return s;
+  if ((s = make_map(&tmQp, q, D, p->hq, p->N + p->T, 1, p->rc)) != SPAVA_OK) return s;
   ScoreParams sp;
   sp.items = all_hosts ? p->d_score_all : p->d_score_pre;
   sp.n_items = n_items;
@@ -345,6 +346,7 @@ spava_status launch_score(const spava_plan* p, const void* q, const void* k, flo
   sp.group = G;
   sp.chunk_tokens = p->rc;
   sp.n_chunks = p->n_chunks;
+  sp.head_reduce = p->score_reduce;
   sp.n_visual = p->N;
   sp.scale = p->scale;
   sp.scores = scores;
@@ -418,6 +420,7 @@ struct TwoStageBufs {
   float* row_o = nullptr;
   float* row_lse = nullptr;
   unsigned int* score_keys = nullptr;
+  int per_qhead = 0;  // score_keys has one row per query head
 };
 
 template <int D>
@@ -459,6 +462,7 @@ spava_status launch_attn(const spava_plan* p, const AttnItem* items, int n_items
   ap.row_o = ts.row_o;
   ap.row_lse = ts.row_lse;
   ap.score_keys = ts.score_keys;
+  ap.score_per_qhead = ts.per_qhead;
   ap.n_visual = p->N;
   ap.probe_r = p->R;
   ap.scale = p->scale;
@@ -594,6 +598,8 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   o = align_up(o + static_cast<size_t>(n_visual) * hq * head_dim * 4, 256);
   p->ws_row_lse = o;
   o = align_up(o + static_cast<size_t>(hq) * n_visual * 4, 256);
+  p->ws_qkeys = o;  // per-query-head score keys (sum / mean head reductions)
+  o = align_up(o + static_cast<size_t>(hq) * n_visual * 4, 256);
   p->ws_total_two_stage = o;
 
   // device
@@ -674,6 +680,14 @@ int32_t spava_plan_offsets(const spava_plan* p, int32_t* offsets_out) {
   if (offsets_out)
     for (int h = 0; h <= p->H; ++h) offsets_out[h] = p->off[h];
   return p->H;
+}
+
+spava_status spava_plan_set_score_reduce(spava_plan* p, int32_t mode) {
+  if (!p) return fail(SPAVA_ERR_INVALID_ARG, "plan is NULL");
+  if (mode != SPAVA_SCORE_MAX && mode != SPAVA_SCORE_SUM && mode != SPAVA_SCORE_MEAN)
+    return fail(SPAVA_ERR_INVALID_ARG, "unknown score reduction %d", mode);
+  p->score_reduce = mode;
+  return ok();
 }
 
 spava_status spava_plan_set_debug(spava_plan* p, uint64_t wait_limit_ns, int32_t stall_producer) {
@@ -814,8 +828,11 @@ spava_status spava_attn_prefill_two_stage(const spava_plan* p, const void* q, co
   TwoStageBufs ts;
   ts.row_o = reinterpret_cast<float*>(w + p->ws_row_o);
   ts.row_lse = reinterpret_cast<float*>(w + p->ws_row_lse);
-  ts.score_keys = reinterpret_cast<unsigned int*>(scores);  // keys, turned into scores in place
-  const size_t n_keys = static_cast<size_t>(p->hkv) * p->N;
+  // Max over heads: one key row per KV head, turned into scores in place.  Sum / mean:
+  // one key row per query head, combined into the scores after the local pass.
+  ts.per_qhead = p->score_reduce != SPAVA_SCORE_MAX;
+  ts.score_keys = ts.per_qhead ? reinterpret_cast<unsigned int*>(w + p->ws_qkeys) : reinterpret_cast<unsigned int*>(scores);
+  const size_t n_keys = static_cast<size_t>(ts.per_qhead ? p->hq : p->hkv) * p->N;
   const int grid_small = std::max(1, std::min(p->num_sms * 4, static_cast<int>((n_keys + 255) / 256)));
   if (scores_needed(*p)) {
     mark(p, kLabFill, st);
@@ -829,7 +846,11 @@ spava_status spava_attn_prefill_two_stage(const spava_plan* p, const void* q, co
   if (s != SPAVA_OK) return s;
   if (scores_needed(*p)) {
     mark(p, kLabFill, st);
-    spava::keys_to_scores_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, n_keys);
+    if (ts.per_qhead)
+      spava::combine_head_keys_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, scores, p->hkv, p->hq / p->hkv,
+                                                                   static_cast<size_t>(p->N), p->score_reduce);
+    else
+      spava::keys_to_scores_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, n_keys);
     SPAVA_CUDA(cudaGetLastError());
     ++g_last_launches;
     if ((s = launch_select(p, scores, idx, st, k, v, kp, vp)) != SPAVA_OK) return s;

@@ -86,3 +86,4 @@ def test_null_arguments(lib):
     assert lib.spava_attn_prefill(None, None, None, None, None, None, None, None, None, None) == \
         _lib.SPAVA_ERR_INVALID_ARG
     assert lib.spava_plan_offsets(None, None) == -1
+    assert lib.spava_plan_set_score_reduce(None, 0) == _lib.SPAVA_ERR_INVALID_ARG
