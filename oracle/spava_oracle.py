@@ -30,7 +30,10 @@ Readings taken where they are silent (each is a parameter of this oracle):
       parity unpinned -- no page value fixes sum vs max.)  Switchable
       (``head_reduce``): with "sum" or "mean" each head first takes its own max
       over the probe rows, m_c(j), and the group's score is sum_c m_c(j) or its
-      mean; "max" is max_c m_c(j), the default above.
+      mean; "max" is max_c m_c(j), the default above.  With "none" every query
+      head keeps its own row m_c(j) and selects its own passing keys (per-query-head
+      selection); query head c then attends to its own passing set, drawn from KV
+      head c // G.
   R2  causal inside the probe: probe row i never scores a key j > i.
   R3  host 0's anchor positions [0, A) are not passing candidates, so no key is
       attended twice by a later host (parity unpinned -- a plan-level reading).
@@ -76,14 +79,15 @@ def _groups(hq: int, hkv: int) -> int:
     return hq // hkv
 
 
-HEAD_REDUCE = ("max", "sum", "mean")
+HEAD_REDUCE = ("max", "sum", "mean", "none")
 
 
 def probe_scores(q: np.ndarray, k: np.ndarray, off: np.ndarray, probe_r: int,
                  scale: float, head_reduce: str = "max") -> np.ndarray:
     """Query-to-context scores of every visual key (readings R1, R2).
 
-    q [tokens, hq, d], k [tokens, hkv, d] float64; returns float64 [hkv, N].
+    q [tokens, hq, d], k [tokens, hkv, d] float64; returns float64 [hkv, N], or
+    [hq, N] (one row per query head, row c = m_c) with head_reduce="none".
     ``head_reduce`` combines the per-head probe maxima of a KV group (R1).
     """
     if head_reduce not in HEAD_REDUCE:
@@ -92,7 +96,7 @@ def probe_scores(q: np.ndarray, k: np.ndarray, off: np.ndarray, probe_r: int,
     G = _groups(hq, hkv)
     H = len(off) - 1
     N = int(off[-1])
-    scores = np.empty((hkv, N), dtype=np.float64)
+    scores = np.empty((hq if head_reduce == "none" else hkv, N), dtype=np.float64)
     for h in range(H):
         a, e = int(off[h]), int(off[h + 1])
         if probe_r > e - a:
@@ -105,7 +109,9 @@ def probe_scores(q: np.ndarray, k: np.ndarray, off: np.ndarray, probe_r: int,
             s = np.matmul(qg.transpose(1, 0, 2), k[a:e, g, :].T)     # [G, R, B]
             s = np.where(visible[None], s * scale, -np.inf)
             per_head = s.max(axis=1)                                 # [G, B]: m_c(j)
-            if head_reduce == "max":
+            if head_reduce == "none":
+                scores[g * G:(g + 1) * G, a:e] = per_head
+            elif head_reduce == "max":
                 scores[g, a:e] = per_head.max(axis=0)
             elif head_reduce == "sum":
                 scores[g, a:e] = per_head.sum(axis=0)
@@ -141,10 +147,21 @@ def select_passing(scores: np.ndarray, off: np.ndarray, anchor: int, passing: in
     return out
 
 
+def sel_row(sel: Optional[np.ndarray], c: int, hq: int, hkv: int) -> int:
+    """Row of the selection that query head c attends through: its KV head c // G when
+    ``sel`` has one row per KV head, c itself when it has one per query head (R1)."""
+    if sel is None or sel.shape[1] == hkv:
+        return c // _groups(hq, hkv)
+    if sel.shape[1] != hq:
+        raise ValueError("selection must have hkv or hq rows")
+    return c
+
+
 def key_set(off: np.ndarray, anchor: int, sel: Optional[np.ndarray], g: int, i: int,
             n_visual: int) -> np.ndarray:
-    """Keys attended by row i through KV head g: anchor | passing of earlier hosts |
-    own block up to i (causal).  Host 0 and text rows: [0, i] (readings R5, R6)."""
+    """Keys attended by row i through selection row g (``sel_row``): anchor | passing
+    of earlier hosts | own block up to i (causal).  Host 0 and text rows: [0, i]
+    (readings R5, R6)."""
     if i >= n_visual:
         return np.arange(0, i + 1)
     h = host_of_row(off, i)
@@ -188,21 +205,22 @@ def approx_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, off: np.ndarra
         a, e = int(off[h]), int(off[h + 1])
         if e <= lo_row or a >= hi_row:
             continue
-        for g in range(hkv):
+        for c in range(hq):
+            g = c // G
             if h == 0:
                 remote = np.zeros(0, dtype=np.int64)
             else:
+                sr = sel_row(sel, c, hq, hkv)
                 remote = np.concatenate([np.arange(0, anchor)] +
-                                        [np.asarray(sel[hp, g], dtype=np.int64) for hp in range(h)])
+                                        [np.asarray(sel[hp, sr], dtype=np.int64) for hp in range(h)])
             for r0 in range(max(a, lo_row), min(e, hi_row), row_chunk):
                 r1 = min(e, hi_row, r0 + row_chunk)
                 keys = np.concatenate([remote, np.arange(a, r1)])
                 visible = np.ones((r1 - r0, keys.size), dtype=bool)
                 visible[:, remote.size:] = np.arange(a, r1)[None, :] <= np.arange(r0, r1)[:, None]
                 kk, vv = k[keys, g, :], v[keys, g, :]
-                for c in range(g * G, (g + 1) * G):
-                    logits = np.matmul(q[r0:r1, c, :], kk.T) * scale
-                    O[r0:r1, c], lse[c, r0:r1] = _masked_softmax_attend(logits, visible, vv)
+                logits = np.matmul(q[r0:r1, c, :], kk.T) * scale
+                O[r0:r1, c], lse[c, r0:r1] = _masked_softmax_attend(logits, visible, vv)
     for r0 in range(max(N, lo_row), min(NT, hi_row), row_chunk):
         r1 = min(NT, hi_row, r0 + row_chunk)
         keys = np.arange(0, r1)
@@ -227,7 +245,7 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, off: np.ndarray,
     L = np.empty(len(rows), dtype=np.float64)
     for n, (i, c) in enumerate(zip(rows, heads)):
         g = int(c) // G
-        keys = key_set(off, anchor, sel, g, int(i), N)
+        keys = key_set(off, anchor, sel, sel_row(sel, int(c), hq, hkv), int(i), N)
         s = np.matmul(k[keys, g, :], q[int(i), int(c), :]) * scale
         m = s.max()
         p = np.exp(s - m)

@@ -177,6 +177,60 @@ def test_blockwise_equals_explicit_mask(H):
             np.testing.assert_allclose(res["lse"][c], (m + np.log(l))[:, 0], rtol=1e-12, atol=1e-12)
 
 
+@pytest.mark.parametrize("H", [2, 4])
+def test_per_query_head_selection_explicit_mask(H):
+    """Per-query-head selection (head_reduce="none"): every query head attends through
+    its own selection row; checked against an explicit mask per query head."""
+    cfg = CONFIGS["tiny"].with_(n_hosts=H, n_text=5, hq=6, hkv=2)
+    g = generate(cfg)
+    q, k, v = (orc.bf16_bits_to_f64(g[x]) for x in ("q", "k", "v"))
+    B = cfg.n_visual // H
+    P = min(cfg.passing, B // 2)
+    A = min(cfg.anchor, B - P)
+    scale = 1 / math.sqrt(cfg.head_dim)
+    res = orc.prefill(q, k, v, g["host_sizes"], A, P, min(cfg.probe_r, B), scale=scale, head_reduce="none")
+    assert res["scores"].shape == (cfg.hq, cfg.n_visual) and res["sel"].shape == (H - 1, cfg.hq, P)
+    off = res["offsets"]
+    G = cfg.hq // cfg.hkv
+    for c in range(cfg.hq):
+        gi = c // G
+        M = _explicit_mask(off, A, res["sel"], c, cfg.n_visual, cfg.n_total)
+        s = q[:, c, :] @ k[:, gi, :].T * scale
+        s = np.where(M, s, -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        p = np.exp(s - m)
+        l = p.sum(axis=1, keepdims=True)
+        np.testing.assert_allclose(res["O"][:, c, :], (p @ v[:, gi, :]) / l, rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(res["lse"][c], (m + np.log(l))[:, 0], rtol=1e-12, atol=1e-12)
+
+
+def test_per_query_head_scores_and_duplicate_heads():
+    """Row c of the per-query-head scores is the max-mode score of the problem made of
+    query head c alone; with every query head of a group a copy of the first, the
+    per-query-head prefill equals the default (max over heads) one."""
+    cfg = CONFIGS["tiny"].with_(n_hosts=4, n_text=3, hq=6, hkv=2)
+    g = generate(cfg)
+    q, k, v = (orc.bf16_bits_to_f64(g[x]) for x in ("q", "k", "v"))
+    off = orc.host_offsets(g["host_sizes"])
+    scale = 1 / math.sqrt(cfg.head_dim)
+    G = cfg.hq // cfg.hkv
+    per = orc.probe_scores(q, k, off, cfg.probe_r, scale, "none")
+    for t in range(G):
+        heads = [gg * G + t for gg in range(cfg.hkv)]
+        np.testing.assert_array_equal(per[heads], orc.probe_scores(q[:, heads], k, off, cfg.probe_r, scale, "max"))
+    qd = q.copy()
+    for gg in range(cfg.hkv):
+        for t in range(1, G):
+            qd[:, gg * G + t] = qd[:, gg * G]
+    a = orc.prefill(qd, k, v, g["host_sizes"], cfg.anchor, cfg.passing, cfg.probe_r, scale=scale)
+    b = orc.prefill(qd, k, v, g["host_sizes"], cfg.anchor, cfg.passing, cfg.probe_r, scale=scale,
+                    head_reduce="none")
+    for c in range(cfg.hq):
+        np.testing.assert_array_equal(b["sel"][:, c], a["sel"][:, c // G])
+    np.testing.assert_allclose(b["O"], a["O"], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(b["lse"], a["lse"], rtol=1e-13, atol=1e-13)
+
+
 def test_rows_formulation_matches_blockwise():
     cfg = CONFIGS["tiny"].with_(n_text=5)
     g = generate(cfg)
