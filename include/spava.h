@@ -29,6 +29,9 @@
  *             idx [H-1][hkv][P] int32, token ids ascending per (host, KV head).
  *             k_pass, v_pass [hkv][H-1][P][d] bf16 (host-major inside a KV head,
  *             so hosts 0..h-1 of one KV head are one contiguous run).
+ *             With SPAVA_SCORE_PER_QUERY_HEAD (spava_plan_set_score_reduce) the
+ *             hkv of scores, idx and k_pass / v_pass becomes hq: one selection
+ *             row per query head.
  *   Pointers  all tensor pointers are DEVICE pointers owned by the caller, 16-byte
  *             aligned; the workspace is 256-byte aligned and at least
  *             spava_workspace_bytes(plan) bytes.  Outputs must not alias inputs.
@@ -103,13 +106,24 @@ spava_status spava_plan_destroy(spava_plan* plan);
  *   SPAVA_SCORE_MAX   score(g, j) = scale * max_c m_c(j)          (default)
  *   SPAVA_SCORE_SUM   score(g, j) = scale * sum_c m_c(j)
  *   SPAVA_SCORE_MEAN  score(g, j) = scale * sum_c m_c(j) / G
- * over the G query heads c of KV head g. */
-typedef enum { SPAVA_SCORE_MAX = 0, SPAVA_SCORE_SUM = 1, SPAVA_SCORE_MEAN = 2 } spava_score_reduce;
+ * over the G query heads c of KV head g, or
+ *   SPAVA_SCORE_PER_QUERY_HEAD  no reduction: score(c, j) = scale * m_c(j) for every
+ *                     query head c, each query head selects its own P passing keys
+ *                     (from KV head c / G) and attends through them.
+ * "Selection rows" below are the hkv KV heads, or the hq query heads in the last mode:
+ * scores [rows, N], indices [H-1, rows, P], passing K/V [rows, H-1, P, d]. */
+typedef enum {
+  SPAVA_SCORE_MAX = 0,
+  SPAVA_SCORE_SUM = 1,
+  SPAVA_SCORE_MEAN = 2,
+  SPAVA_SCORE_PER_QUERY_HEAD = 3
+} spava_score_reduce;
 
 /* Select the head reduction (spava_score_reduce) for this plan's later calls
- * (spava_score_select, spava_attn_prefill and its variants).  Host-side only; the
- * workspace sizes do not depend on it.  Returns SPAVA_ERR_INVALID_ARG for a NULL plan
- * or an unknown mode. */
+ * (spava_score_select, spava_gather_passing, spava_attn_prefill and its variants).
+ * Host-side only.  It sets the number of selection rows, so query
+ * spava_workspace_bytes / spava_two_stage_workspace_bytes after it.  Returns
+ * SPAVA_ERR_INVALID_ARG for a NULL plan or an unknown mode. */
 spava_status spava_plan_set_score_reduce(spava_plan* plan, int32_t mode);
 
 /* Bytes of scratch the calls below need (scores, indices, passing K/V, text

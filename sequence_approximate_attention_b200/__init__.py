@@ -86,15 +86,19 @@ class Plan:
         n = self.two_stage_workspace_bytes if two_stage else self.workspace_bytes
         return torch.zeros(max(n, 256), dtype=torch.uint8, device=self.device)
 
-    SCORE_REDUCE = {"max": 0, "sum": 1, "mean": 2}
+    SCORE_REDUCE = {"max": 0, "sum": 1, "mean": 2, "per_query_head": 3}
 
     def set_score_reduce(self, mode: str) -> None:
         """spava_plan_set_score_reduce: how the query heads of a KV group combine the
-        probe scores ("max" default, "sum", "mean" of the per-head maxima)."""
+        probe scores ("max" default, "sum", "mean" of the per-head maxima), or
+        "per_query_head": every query head selects its own passing keys.  Call before
+        new_workspace: the selection rows set the workspace size."""
         if mode not in self.SCORE_REDUCE:
             raise ValueError(f"score reduction must be one of {sorted(self.SCORE_REDUCE)}")
         _lib.check(self.lib.spava_plan_set_score_reduce(self._h, self.SCORE_REDUCE[mode]), "spava_plan_set_score_reduce")
         self.score_reduce = mode
+        self.workspace_bytes = int(self.lib.spava_workspace_bytes(self._h))
+        self.two_stage_workspace_bytes = int(self.lib.spava_two_stage_workspace_bytes(self._h))
 
     def set_debug(self, wait_limit_ns: int = 0, stall_producer: bool = False) -> None:
         _lib.check(self.lib.spava_plan_set_debug(self._h, int(wait_limit_ns), int(bool(stall_producer))),
@@ -132,11 +136,19 @@ class Plan:
         NT = self.n_total
         return (NT, self.hq, self.head_dim), (NT, self.hkv, self.head_dim)
 
+    @property
+    def score_rows(self) -> int:
+        """Selection rows: KV heads, or query heads with per-query-head selection."""
+        return self.hq if getattr(self, "score_reduce", "max") == "per_query_head" else self.hkv
+
+    def scores_shape(self):
+        return (self.score_rows, self.n_visual)
+
     def idx_shape(self):
-        return (max(self.n_hosts - 1, 0), self.hkv, self.passing)
+        return (max(self.n_hosts - 1, 0), self.score_rows, self.passing)
 
     def pass_shape(self):
-        return (self.hkv, max(self.n_hosts - 1, 0), self.passing, self.head_dim)
+        return (self.score_rows, max(self.n_hosts - 1, 0), self.passing, self.head_dim)
 
     def _check_qkv(self, q, k, v=None):
         qs, ks = self.qkv_shapes()
@@ -162,12 +174,12 @@ def score_select(plan: Plan, q: Optional[torch.Tensor], k: Optional[torch.Tensor
     """spava_score_select: probe scores [hkv, N] fp32 and passing indices [H-1, hkv, P]."""
     dev = plan.device
     if scores_given:
-        _expect(scores, "scores", torch.float32, (plan.hkv, plan.n_visual), dev)
+        _expect(scores, "scores", torch.float32, plan.scores_shape(), dev)
     else:
         plan._check_qkv(q, k)
         if scores is None:
-            scores = torch.empty((plan.hkv, plan.n_visual), dtype=torch.float32, device=dev)
-        _expect(scores, "scores", torch.float32, (plan.hkv, plan.n_visual), dev)
+            scores = torch.empty(plan.scores_shape(), dtype=torch.float32, device=dev)
+        _expect(scores, "scores", torch.float32, plan.scores_shape(), dev)
     if idx is None:
         idx = torch.empty(plan.idx_shape(), dtype=torch.int32, device=dev)
     _expect(idx, "idx", torch.int32, plan.idx_shape(), dev)
@@ -215,7 +227,7 @@ def attn_prefill(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     _expect(o, "o", torch.bfloat16, tuple(q.shape), dev)
     _expect(lse, "lse", torch.float32, (plan.hq, plan.n_total), dev)
     if scores_out is not None:
-        _expect(scores_out, "scores_out", torch.float32, (plan.hkv, plan.n_visual), dev)
+        _expect(scores_out, "scores_out", torch.float32, plan.scores_shape(), dev)
     if idx_out is not None:
         _expect(idx_out, "idx_out", torch.int32, plan.idx_shape(), dev)
     ws = _ws(plan, workspace)
@@ -241,7 +253,7 @@ def attn_prefill_two_stage(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torc
     _expect(o, "o", torch.bfloat16, tuple(q.shape), dev)
     _expect(lse, "lse", torch.float32, (plan.hq, plan.n_total), dev)
     if scores_out is not None:
-        _expect(scores_out, "scores_out", torch.float32, (plan.hkv, plan.n_visual), dev)
+        _expect(scores_out, "scores_out", torch.float32, plan.scores_shape(), dev)
     if idx_out is not None:
         _expect(idx_out, "idx_out", torch.int32, plan.idx_shape(), dev)
     ws = _ws(plan, workspace, two_stage=True)

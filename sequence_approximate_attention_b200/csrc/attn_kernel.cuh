@@ -67,6 +67,7 @@ struct AttnParams {
   const AttnItem* items;
   int n_items;
   int group;       // hq / hkv
+  int pass_per_qhead;  // passing buffers have one row per query head (per-query-head selection)
   int hq;
   int n_rows_out;  // rows of o and lse (N + T)
   __nv_bfloat16* o;
@@ -291,7 +292,8 @@ __global__ void __launch_bounds__(384, 1)
               const CUtensorMap* map = passing ? (kv ? &tmVp : &tmKp) : (kv ? &tmV : &tmK);
               for (int hh = 0; hh < S::kHalves; ++hh) {
                 if (passing)
-                  tma_load_3d(dst + hh * S::kHalfBytes, map, kv_full + slot, hh * 64, row, kvh);
+                  tma_load_3d(dst + hh * S::kHalfBytes, map, kv_full + slot, hh * 64, row,
+                              p.pass_per_qhead ? it.q_head : kvh);
                 else
                   tma_load_3d(dst + hh * S::kHalfBytes, map, kv_full + slot, hh * 64, kvh, row);
               }

@@ -5,7 +5,8 @@
 //   m_c(j)   = max over probe rows i in [e-R, e), i >= j, of (q_{i,c} . k_{j,g})
 //   score(g, j) = scale * reduce over the query heads c of group g of m_c(j),
 //   e = end of j's host block; reduce = max (default), sum or mean (the pages leave
-//   the combination open; max over heads and rows is the plainest reading).
+//   the combination open; max over heads and rows is the plainest reading), or none:
+//   one score row m_c per query head (per-query-head selection).
 //
 // The product is computed transposed, S^T = K_tile * Qprobe^T, so that each TMEM
 // lane holds one key and the max over (probe row, head) is a per-thread reduction
@@ -31,7 +32,8 @@ struct ScoreParams {
   int group;         // G = hq / hkv
   int chunk_tokens;  // Rc probe tokens per N chunk (Rc * G <= 256, multiple of 16)
   int n_chunks;      // ceil(R / Rc)
-  int head_reduce;   // 0 max, 1 sum, 2 mean over the group's query heads
+  int head_reduce;   // 0 max, 1 sum, 2 mean over the group's query heads; 3 none (one
+                     // score row per query head: scores is [hq][N])
   int n_visual;      // N (row stride of scores)
   float scale;
   float* scores;     // [hkv][N]
@@ -330,6 +332,14 @@ __global__ void __launch_bounds__(256, 1)
         if (lane == 0) mbar_arrive(acc_empty + b);
       }
       if (!ok) break;
+      if (p.head_reduce == 3) {
+        if (j < e) {
+#pragma unroll 1
+          for (int h = 0; h < G; ++h)
+            p.scores[(static_cast<size_t>(it.y) * G + h) * p.n_visual + j] = mh[h] * p.scale;
+        }
+        continue;
+      }
       float r = mx_all;
       if (by_head) {
         r = 0.f;

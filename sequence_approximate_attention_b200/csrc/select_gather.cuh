@@ -37,7 +37,8 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
   return res;
 }
 
-// One CTA per (host h < H-1, KV head g).  Candidates: [off[h] + (h == 0 ? A : 0),
+// One CTA per (host h < H-1, selection row g: a KV head, or a query head with
+// per-query-head selection).  Candidates: [off[h] + (h == 0 ? A : 0),
 // off[h+1]).  Radix select (four 8-bit digits, most significant first) finds the
 // P-th largest key T and how many keys equal to T are taken; a stable compaction in
 // index order then writes the P winners ascending: keys > T, and the lowest-index
@@ -56,20 +57,22 @@ struct GatherArgs {
   uint4* vp;
   int hosts_m1;
   int chunks_per_row;  // 16-byte chunks per K/V row (d * 2 / 16)
+  int kv_heads;        // hkv (row stride of k and v)
+  int group_div;       // selection row r reads KV head r / group_div (1, or G per query head)
 };
 
 template <int kPer, bool kGather>
 __global__ void __launch_bounds__(1024) select_topp_kernel(const float* __restrict__ scores, int n_visual,
                                                             const int* __restrict__ off, int anchor, int passing,
-                                                            int hkv, int32_t* __restrict__ idx, GatherArgs ga) {
+                                                            int rows, int32_t* __restrict__ idx, GatherArgs ga) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t scan_scratch[33];
   __shared__ uint32_t sh_prefix, sh_k;
-  const int h = blockIdx.x / hkv, g = blockIdx.x % hkv;
+  const int h = blockIdx.x / rows, g = blockIdx.x % rows;
   const int lo = off[h] + (h == 0 ? anchor : 0), hi = off[h + 1];
   const int n = hi - lo;
   const float* s = scores + static_cast<size_t>(g) * n_visual + lo;
-  int32_t* out = idx + (static_cast<size_t>(h) * hkv + g) * passing;
+  int32_t* out = idx + (static_cast<size_t>(h) * rows + g) * passing;
   const int tid = threadIdx.x, nt = blockDim.x;
   if (passing <= 0) return;
   const int per = (n + nt - 1) / nt;
@@ -166,6 +169,7 @@ __global__ void __launch_bounds__(1024) select_topp_kernel(const float* __restri
     const int cpr_shift = __ffs(cpr) - 1;
     const int total = passing * cpr;
     const size_t dst0 = ((static_cast<size_t>(g) * ga.hosts_m1 + h) * passing) * cpr;
+    const int kvh = g / ga.group_div;
     for (int t0 = tid; t0 < total; t0 += kGatherUnroll * nt) {
       uint4 kv[kGatherUnroll], vv[kGatherUnroll];
 #pragma unroll
@@ -173,7 +177,7 @@ __global__ void __launch_bounds__(1024) select_topp_kernel(const float* __restri
         const int t = t0 + u * nt;
         if (t < total) {
           const int r = t >> cpr_shift, ch = t & (cpr - 1);
-          const size_t src = (static_cast<size_t>(out[r]) * hkv + g) * cpr + ch;
+          const size_t src = (static_cast<size_t>(out[r]) * ga.kv_heads + kvh) * cpr + ch;
           kv[u] = __ldg(ga.k + src);
           vv[u] = __ldg(ga.v + src);
         }
@@ -219,13 +223,15 @@ __global__ void __launch_bounds__(256) combine_head_keys_kernel(const uint32_t* 
   }
 }
 
-// k_pass[g][h][j][:] = k[idx[h][g][j]][g][:] (same for v), 16 bytes per thread.
+// k_pass[g][h][j][:] = k[idx[h][g][j]][g / group_div][:] (same for v), 16 bytes per
+// thread; g runs over the selection rows (KV heads, or query heads).
 __global__ void __launch_bounds__(256) gather_passing_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                                               const int32_t* __restrict__ idx, uint4* __restrict__ kp,
-                                                              uint4* __restrict__ vp, int hkv, int hosts_m1,
-                                                              int passing, int chunks_per_row) {
+                                                              uint4* __restrict__ vp, int rows, int kv_heads,
+                                                              int group_div, int hosts_m1, int passing,
+                                                              int chunks_per_row) {
   const size_t rows_per_g = static_cast<size_t>(hosts_m1) * passing;
-  const size_t total = static_cast<size_t>(hkv) * rows_per_g * chunks_per_row;
+  const size_t total = static_cast<size_t>(rows) * rows_per_g * chunks_per_row;
   for (size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
        t += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const size_t r = t / chunks_per_row;
@@ -234,8 +240,8 @@ __global__ void __launch_bounds__(256) gather_passing_kernel(const uint4* __rest
     const size_t rem = r - static_cast<size_t>(g) * rows_per_g;
     const int h = static_cast<int>(rem / passing);
     const int j = static_cast<int>(rem - static_cast<size_t>(h) * passing);
-    const int tok = __ldg(idx + (static_cast<size_t>(h) * hkv + g) * passing + j);
-    const size_t src = (static_cast<size_t>(tok) * hkv + g) * chunks_per_row + ch;
+    const int tok = __ldg(idx + (static_cast<size_t>(h) * rows + g) * passing + j);
+    const size_t src = (static_cast<size_t>(tok) * kv_heads + g / group_div) * chunks_per_row + ch;
     kp[t] = __ldg(k + src);
     vp[t] = __ldg(v + src);
   }

@@ -321,6 +321,41 @@ unsigned int* err_word(const spava_plan* p, void* ws) {
   return reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + p->ws_err);
 }
 
+// Rows of scores, selections and passing buffers: one per KV head, or one per query
+// head with per-query-head selection.
+int score_rows(const spava_plan& p) { return p.score_reduce == SPAVA_SCORE_PER_QUERY_HEAD ? p.hq : p.hkv; }
+
+// Byte offsets of the workspace (sized by the plan and by the selection rows).
+void layout_workspace(spava_plan* p) {
+  const size_t n_visual = static_cast<size_t>(p->N), n_text = static_cast<size_t>(p->T);
+  const size_t hq = static_cast<size_t>(p->hq), d = static_cast<size_t>(p->d), P = static_cast<size_t>(p->P);
+  const size_t rows = static_cast<size_t>(score_rows(*p));
+  const size_t hm1 = p->H > 1 ? static_cast<size_t>(p->H - 1) : 0;
+  size_t o = 0;
+  p->ws_err = o;
+  o += 256;
+  p->ws_scores = o;
+  o = align_up(o + rows * n_visual * 4, 256);
+  p->ws_idx = o;
+  o = align_up(o + hm1 * rows * P * 4, 256);
+  p->ws_kp = o;
+  o = align_up(o + hm1 * rows * P * d * 2, 256);
+  p->ws_vp = o;
+  o = align_up(o + hm1 * rows * P * d * 2, 256);
+  p->ws_opart = o;
+  o = align_up(o + static_cast<size_t>(p->H + 1) * n_text * hq * d * 4, 256);
+  p->ws_lpart = o;
+  o = align_up(o + static_cast<size_t>(p->H + 1) * hq * n_text * 4, 256);
+  p->ws_total = o;
+  p->ws_row_o = o;
+  o = align_up(o + n_visual * hq * d * 4, 256);
+  p->ws_row_lse = o;
+  o = align_up(o + hq * n_visual * 4, 256);
+  p->ws_qkeys = o;  // per-query-head score keys (all but the max head reduction)
+  o = align_up(o + hq * n_visual * 4, 256);
+  p->ws_total_two_stage = o;
+}
+
 spava_status check_plan_ws(const spava_plan* p, void* ws) {
   if (!p) return fail(SPAVA_ERR_INVALID_ARG, "plan is NULL");
   if (!ws) return fail(SPAVA_ERR_INVALID_ARG, "workspace is NULL");
@@ -379,21 +414,22 @@ spava_status launch_select(const spava_plan* p, const float* scores, int32_t* id
   if (p->H < 2 || p->P == 0) return SPAVA_OK;
   int max_seg = 0;
   for (int h = 0; h + 1 < p->H; ++h) max_seg = std::max(max_seg, p->off[h + 1] - p->off[h]);
+  const int rows = score_rows(*p);
   spava::GatherArgs ga{static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(kp),
-                       static_cast<uint4*>(vp), p->H - 1, p->d * 2 / 16};
+                       static_cast<uint4*>(vp), p->H - 1, p->d * 2 / 16, p->hkv, rows / p->hkv};
   const bool fused = k != nullptr;
-  const int grid = (p->H - 1) * p->hkv;
+  const int grid = (p->H - 1) * rows;
   mark(p, fused ? kLabSelectGather : kLabSelect, st);
   if (max_seg <= 16 * 1024) {
     if (fused)
-      spava::select_topp_kernel<16, true><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, p->hkv, idx, ga);
+      spava::select_topp_kernel<16, true><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, rows, idx, ga);
     else
-      spava::select_topp_kernel<16, false><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, p->hkv, idx, ga);
+      spava::select_topp_kernel<16, false><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, rows, idx, ga);
   } else {
     if (fused)
-      spava::select_topp_kernel<0, true><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, p->hkv, idx, ga);
+      spava::select_topp_kernel<0, true><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, rows, idx, ga);
     else
-      spava::select_topp_kernel<0, false><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, p->hkv, idx, ga);
+      spava::select_topp_kernel<0, false><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, rows, idx, ga);
   }
   SPAVA_CUDA(cudaGetLastError());
   ++g_last_launches;
@@ -404,12 +440,13 @@ spava_status launch_gather(const spava_plan* p, const void* k, const void* v, co
                            cudaStream_t st) {
   if (p->H < 2 || p->P == 0) return SPAVA_OK;
   const int chunks = p->d * 2 / 16;
-  const size_t total = static_cast<size_t>(p->hkv) * (p->H - 1) * p->P * chunks;
+  const int rows = score_rows(*p);
+  const size_t total = static_cast<size_t>(rows) * (p->H - 1) * p->P * chunks;
   const int grid = static_cast<int>(std::min<size_t>((total + 255) / 256, static_cast<size_t>(p->num_sms) * 8));
   mark(p, kLabGather, st);
   spava::gather_passing_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), idx,
-                                                      static_cast<uint4*>(kp), static_cast<uint4*>(vp), p->hkv,
-                                                      p->H - 1, p->P, chunks);
+                                                      static_cast<uint4*>(kp), static_cast<uint4*>(vp), rows, p->hkv,
+                                                      rows / p->hkv, p->H - 1, p->P, chunks);
   SPAVA_CUDA(cudaGetLastError());
   ++g_last_launches;
   return SPAVA_OK;
@@ -436,8 +473,8 @@ spava_status launch_attn(const spava_plan* p, const AttnItem* items, int n_items
   if ((s = make_map(&tmV, v, D, p->hkv, NT, 1, 128)) != SPAVA_OK) return s;
   if (p->H >= 2 && p->P > 0 && kp && vp) {
     const uint64_t rows = static_cast<uint64_t>(p->H - 1) * p->P;
-    if ((s = make_map(&tmKp, kp, D, rows, p->hkv, 128, 1)) != SPAVA_OK) return s;
-    if ((s = make_map(&tmVp, vp, D, rows, p->hkv, 128, 1)) != SPAVA_OK) return s;
+    if ((s = make_map(&tmKp, kp, D, rows, score_rows(*p), 128, 1)) != SPAVA_OK) return s;
+    if ((s = make_map(&tmVp, vp, D, rows, score_rows(*p), 128, 1)) != SPAVA_OK) return s;
   } else {
     tmKp = tmK;  // never read: no item has a passing segment
     tmVp = tmV;
@@ -446,6 +483,7 @@ spava_status launch_attn(const spava_plan* p, const AttnItem* items, int n_items
   ap.items = items;
   ap.n_items = n_items;
   ap.group = p->hq / p->hkv;
+  ap.pass_per_qhead = p->score_reduce == SPAVA_SCORE_PER_QUERY_HEAD;
   ap.hq = p->hq;
   ap.n_rows_out = p->N + p->T;
   ap.o = static_cast<__nv_bfloat16*>(o);
@@ -576,31 +614,7 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   if (probe_r > 0) p->rc = std::min(p->rc, probe_r);
   p->n_chunks = probe_r > 0 ? ceil_div(probe_r, p->rc) : 0;
 
-  // workspace layout
-  size_t o = 0;
-  p->ws_err = o;
-  o += 256;
-  p->ws_scores = o;
-  o = align_up(o + static_cast<size_t>(hkv) * n_visual * 4, 256);
-  const size_t hm1 = n_hosts > 1 ? n_hosts - 1 : 0;
-  p->ws_idx = o;
-  o = align_up(o + hm1 * hkv * passing * 4, 256);
-  p->ws_kp = o;
-  o = align_up(o + hm1 * hkv * passing * head_dim * 2, 256);
-  p->ws_vp = o;
-  o = align_up(o + hm1 * hkv * passing * head_dim * 2, 256);
-  p->ws_opart = o;
-  o = align_up(o + static_cast<size_t>(n_hosts + 1) * n_text * hq * head_dim * 4, 256);
-  p->ws_lpart = o;
-  o = align_up(o + static_cast<size_t>(n_hosts + 1) * hq * n_text * 4, 256);
-  p->ws_total = o;
-  p->ws_row_o = o;
-  o = align_up(o + static_cast<size_t>(n_visual) * hq * head_dim * 4, 256);
-  p->ws_row_lse = o;
-  o = align_up(o + static_cast<size_t>(hq) * n_visual * 4, 256);
-  p->ws_qkeys = o;  // per-query-head score keys (sum / mean head reductions)
-  o = align_up(o + static_cast<size_t>(hq) * n_visual * 4, 256);
-  p->ws_total_two_stage = o;
+  layout_workspace(p);
 
   // device
   auto bail = [&](spava_status s) {
@@ -684,9 +698,11 @@ int32_t spava_plan_offsets(const spava_plan* p, int32_t* offsets_out) {
 
 spava_status spava_plan_set_score_reduce(spava_plan* p, int32_t mode) {
   if (!p) return fail(SPAVA_ERR_INVALID_ARG, "plan is NULL");
-  if (mode != SPAVA_SCORE_MAX && mode != SPAVA_SCORE_SUM && mode != SPAVA_SCORE_MEAN)
+  if (mode != SPAVA_SCORE_MAX && mode != SPAVA_SCORE_SUM && mode != SPAVA_SCORE_MEAN &&
+      mode != SPAVA_SCORE_PER_QUERY_HEAD)
     return fail(SPAVA_ERR_INVALID_ARG, "unknown score reduction %d", mode);
   p->score_reduce = mode;
+  layout_workspace(p);  // selection rows decide the sizes of scores, indices, passing K/V
   return ok();
 }
 
@@ -846,7 +862,10 @@ spava_status spava_attn_prefill_two_stage(const spava_plan* p, const void* q, co
   if (s != SPAVA_OK) return s;
   if (scores_needed(*p)) {
     mark(p, kLabFill, st);
-    if (ts.per_qhead)
+    if (p->score_reduce == SPAVA_SCORE_PER_QUERY_HEAD)  // one score row per query head: convert
+      spava::combine_head_keys_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, scores, p->hq, 1,
+                                                                   static_cast<size_t>(p->N), SPAVA_SCORE_SUM);
+    else if (ts.per_qhead)
       spava::combine_head_keys_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, scores, p->hkv, p->hq / p->hkv,
                                                                    static_cast<size_t>(p->N), p->score_reduce);
     else

@@ -1,5 +1,6 @@
 """GPU parity of the switchable head reduction of the probe scores (sum and mean of the
-per-head maxima beside the default max), through spava_plan_set_score_reduce.
+per-head maxima beside the default max, and per-query-head selection), through
+spava_plan_set_score_reduce.
 
 Standalone scoring (spava_score_select) and both prefill flows (the score kernel, and
 the fused local-pass scores of the two-stage flow) against the fp64 oracle with the
@@ -46,13 +47,16 @@ def _setup(name, mode):
     plan.set_score_reduce(mode)
     off = orc.host_offsets(sizes)
     scale = 1.0 / math.sqrt(cfg.head_dim)
-    ref = orc.probe_scores(f64["q"], f64["k"], off, cfg.probe_r, scale, head_reduce=mode)
+    per_head = mode == "per_query_head"
+    ref = orc.probe_scores(f64["q"], f64["k"], off, cfg.probe_r, scale, head_reduce="none" if per_head else mode)
     G = cfg.hq // cfg.hkv
     tol = score_tolerance(f64["q"], f64["k"], off, cfg.probe_r, scale) * (G if mode == "sum" else 1)
+    if per_head:
+        tol = np.repeat(tol, G, axis=0)   # the group's bound holds for each of its heads
     return cfg, f64, dev, plan, off, scale, ref, tol
 
 
-@pytest.mark.parametrize("mode", ["sum", "mean"])
+@pytest.mark.parametrize("mode", ["sum", "mean", "per_query_head"])
 @pytest.mark.parametrize("name", list(CASES))
 def test_score_select_head_reduce(name, mode):
     cfg, f64, dev, plan, off, scale, ref, tol = _setup(name, mode)
@@ -66,12 +70,12 @@ def test_score_select_head_reduce(name, mode):
 
 
 @pytest.mark.parametrize("two_stage", [False, True])
-@pytest.mark.parametrize("mode", ["sum", "mean"])
+@pytest.mark.parametrize("mode", ["sum", "mean", "per_query_head"])
 @pytest.mark.parametrize("name", list(CASES))
 def test_prefill_head_reduce(name, mode, two_stage):
     cfg, f64, dev, plan, off, scale, ref, tol = _setup(name, mode)
     ws = plan.new_workspace(two_stage=two_stage)
-    scores = torch.full((cfg.hkv, cfg.n_visual), float("nan"), device="cuda")
+    scores = torch.full(plan.scores_shape(), float("nan"), device="cuda")
     idx = torch.full(plan.idx_shape(), -1, dtype=torch.int32, device="cuda")
     prefill = sab.attn_prefill_two_stage if two_stage else sab.attn_prefill
     o, lse = prefill(plan, dev["q"], dev["k"], dev["v"], scores_out=scores, idx_out=idx, workspace=ws)
@@ -96,4 +100,25 @@ def test_unknown_mode_is_refused():
     with pytest.raises(ValueError):
         plan.set_score_reduce("median")
     assert plan.lib.spava_plan_set_score_reduce(plan.handle, 7) == 1   # SPAVA_ERR_INVALID_ARG
+    plan.close()
+
+
+@pytest.mark.parametrize("name", ["tiny", "d128_g7_uneven"])
+def test_gather_per_query_head(name):
+    """Standalone gather with one selection row per query head: k_pass[c][h][j] =
+    k[idx[h][c][j]][c // G], byte for byte."""
+    cfg, f64, dev, plan, off, scale, ref, tol = _setup(name, "per_query_head")
+    G = cfg.hq // cfg.hkv
+    scores, idx = sab.score_select(plan, dev["q"], dev["k"])
+    kp, vp = sab.gather_passing(plan, dev["k"], dev["v"], idx)
+    torch.cuda.synchronize()
+    idx_h = idx.cpu().numpy()
+    k16, v16 = dev["k"].cpu().view(torch.int16), dev["v"].cpu().view(torch.int16)
+    kp16, vp16 = kp.cpu().view(torch.int16), vp.cpu().view(torch.int16)
+    assert kp.shape == (cfg.hq, cfg.n_hosts - 1, cfg.passing, cfg.head_dim)
+    for c in range(cfg.hq):
+        for h in range(cfg.n_hosts - 1):
+            rows = torch.from_numpy(idx_h[h, c].astype(np.int64))
+            assert torch.equal(kp16[c, h], k16[rows, c // G]), (name, c, h)
+            assert torch.equal(vp16[c, h], v16[rows, c // G]), (name, c, h)
     plan.close()
