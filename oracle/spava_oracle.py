@@ -33,7 +33,11 @@ Readings taken where they are silent (each is a parameter of this oracle):
       mean; "max" is max_c m_c(j), the default above.  With "none" every query
       head keeps its own row m_c(j) and selects its own passing keys (per-query-head
       selection); query head c then attends to its own passing set, drawn from KV
-      head c // G.
+      head c // G.  ``score_kind`` "prob" replaces each logit by the probe row's
+      attention probability over its own host block, p_c(i, j) = exp(s_c(i, j) -
+      lse_c(i)) with lse_c(i) = log sum over keys j' of the block, j' <= i, of
+      exp s_c(i, j'); m_c(j) is then the max of p_c over the probe rows (the pages'
+      scores may be read as the attention weights rather than the logits).
   R2  causal inside the probe: probe row i never scores a key j > i.
   R3  host 0's anchor positions [0, A) are not passing candidates, so no key is
       attended twice by a later host (parity unpinned -- a plan-level reading).
@@ -80,10 +84,11 @@ def _groups(hq: int, hkv: int) -> int:
 
 
 HEAD_REDUCE = ("max", "sum", "mean", "none")
+SCORE_KIND = ("logit", "prob")
 
 
 def probe_scores(q: np.ndarray, k: np.ndarray, off: np.ndarray, probe_r: int,
-                 scale: float, head_reduce: str = "max") -> np.ndarray:
+                 scale: float, head_reduce: str = "max", score_kind: str = "logit") -> np.ndarray:
     """Query-to-context scores of every visual key (readings R1, R2).
 
     q [tokens, hq, d], k [tokens, hkv, d] float64; returns float64 [hkv, N], or
@@ -92,6 +97,8 @@ def probe_scores(q: np.ndarray, k: np.ndarray, off: np.ndarray, probe_r: int,
     """
     if head_reduce not in HEAD_REDUCE:
         raise ValueError(f"head_reduce must be one of {HEAD_REDUCE}")
+    if score_kind not in SCORE_KIND:
+        raise ValueError(f"score_kind must be one of {SCORE_KIND}")
     hq, hkv = q.shape[1], k.shape[1]
     G = _groups(hq, hkv)
     H = len(off) - 1
@@ -108,6 +115,11 @@ def probe_scores(q: np.ndarray, k: np.ndarray, off: np.ndarray, probe_r: int,
             qg = q[e - probe_r:e, g * G:(g + 1) * G, :]              # [R, G, d]
             s = np.matmul(qg.transpose(1, 0, 2), k[a:e, g, :].T)     # [G, R, B]
             s = np.where(visible[None], s * scale, -np.inf)
+            if score_kind == "prob":
+                # each probe row's softmax over the keys of its block it can see
+                mrow = s.max(axis=2, keepdims=True)
+                lse = mrow + np.log(np.exp(s - mrow).sum(axis=2, keepdims=True))
+                s = np.exp(s - lse)                                  # 0 where not visible
             per_head = s.max(axis=1)                                 # [G, B]: m_c(j)
             if head_reduce == "none":
                 scores[g * G:(g + 1) * G, a:e] = per_head
@@ -284,7 +296,8 @@ def lse_merge(o1: np.ndarray, l1: np.ndarray, o2: np.ndarray, l2: np.ndarray):
 
 def prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, host_sizes: Sequence[int],
             anchor: int, passing: int, probe_r: int, scale: Optional[float] = None,
-            sel: Optional[np.ndarray] = None, rows=None, head_reduce: str = "max") -> Dict[str, np.ndarray]:
+            sel: Optional[np.ndarray] = None, rows=None, head_reduce: str = "max",
+            score_kind: str = "logit") -> Dict[str, np.ndarray]:
     """Whole prefill: split -> score -> select -> approximate attention.
 
     q/k/v are float64 (see ``bf16_bits_to_f64``).  If ``sel`` is given it replaces
@@ -296,7 +309,7 @@ def prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, host_sizes: Sequence[in
         scale = 1.0 / np.sqrt(d)
     off = host_offsets(host_sizes)
     out: Dict[str, np.ndarray] = {"offsets": off}
-    out["scores"] = probe_scores(q, k, off, probe_r, scale, head_reduce)
+    out["scores"] = probe_scores(q, k, off, probe_r, scale, head_reduce, score_kind)
     out["sel"] = select_passing(out["scores"], off, anchor, passing) if sel is None else sel
     if rows is None:
         out["O"], out["lse"] = approx_attention(q, k, v, off, anchor, out["sel"], scale)

@@ -339,6 +339,56 @@ def test_scores_head_reduce_decomposes_over_heads():
         orc.probe_scores(q, k, off, cfg.probe_r, scale, "median")
 
 
+@pytest.mark.parametrize("mode", ["max", "sum"])
+def test_prob_scores_brute_force(mode):
+    """score_kind="prob": each probe row's softmax over the block keys it sees, then
+    the max over probe rows and the head reduction -- pure-Python loops."""
+    rng = np.random.default_rng(6)
+    sizes = [10, 13, 9]
+    hq, hkv, d, R = 4, 2, 3, 4
+    q, k, _ = _rand_qkv(rng, sum(sizes), hq, hkv, d)
+    scale = 0.8
+    off = orc.host_offsets(sizes)
+    got = orc.probe_scores(q, k, off, R, scale, head_reduce=mode, score_kind="prob")
+    G = hq // hkv
+    for h in range(len(sizes)):
+        a, e = int(off[h]), int(off[h + 1])
+        for g in range(hkv):
+            for j in range(a, e):
+                per = []
+                for c in range(g * G, (g + 1) * G):
+                    best = 0.0
+                    for i in range(max(j, e - R), e):
+                        logit = [sum(q[i, c, t] * k[jj, g, t] for t in range(d)) * scale for jj in range(a, i + 1)]
+                        z = sum(math.exp(x - max(logit)) for x in logit)
+                        best = max(best, math.exp(logit[j - a] - max(logit)) / z)
+                    per.append(best)
+                want = max(per) if mode == "max" else sum(per)
+                assert got[g, j] == pytest.approx(want, rel=1e-12, abs=1e-15)
+
+
+def test_prob_scores_invariants():
+    """Probabilities: within (0, 1]; for every head the scores of a host's keys add up
+    to at least 1 (they dominate the last probe row's distribution); with one probe row
+    the selection equals the logit selection (a monotone map of the same row)."""
+    cfg = CONFIGS["tiny"].with_(n_hosts=4, hq=4, hkv=2)
+    g = generate(cfg)
+    q, k = orc.bf16_bits_to_f64(g["q"]), orc.bf16_bits_to_f64(g["k"])
+    off = orc.host_offsets(g["host_sizes"])
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    per = orc.probe_scores(q, k, off, cfg.probe_r, scale, "none", "prob")
+    assert (per > 0).all() and (per <= 1 + 1e-12).all()
+    for h in range(cfg.n_hosts):
+        a, e = int(off[h]), int(off[h + 1])
+        assert (per[:, a:e].sum(axis=1) >= 1 - 1e-12).all()
+    sp = orc.probe_scores(q, k, off, 1, scale, "none", "prob")
+    sl = orc.probe_scores(q, k, off, 1, scale, "none", "logit")
+    np.testing.assert_array_equal(orc.select_passing(sp, off, cfg.anchor, cfg.passing),
+                                  orc.select_passing(sl, off, cfg.anchor, cfg.passing))
+    with pytest.raises(ValueError):
+        orc.probe_scores(q, k, off, cfg.probe_r, scale, "max", "softmax")
+
+
 def _brute_select(vals, lo, P):
     order = sorted(range(len(vals)), key=lambda t: (-float(vals[t]), t))
     return sorted(lo + t for t in order[:P])
