@@ -126,6 +126,25 @@ typedef enum {
  * SPAVA_ERR_INVALID_ARG for a NULL plan or an unknown mode. */
 spava_status spava_plan_set_score_reduce(spava_plan* plan, int32_t mode);
 
+/* What a probe row contributes to a key's score (the same passage leaves it open
+ * whether the attention scores are the logits or the attention weights):
+ *   SPAVA_SCORE_LOGIT  q_{i,c} . k_j (scaled), as above               (default)
+ *   SPAVA_SCORE_PROB   exp(scale * q_{i,c} . k_j - lse_c(i)): the probe row's
+ *                      attention probability over the keys of its own host block
+ *                      it sees (lse_c(i) = log sum over keys j' <= i of the block of
+ *                      exp(scale * q_{i,c} . k_j'), computed by the attention kernel
+ *                      over the probe rows first); m_c(j) is the max of these over
+ *                      the probe rows, then the head reduction applies as above.
+ * The two-stage flow scores with the score kernel in this mode (the final lse of a
+ * probe row is not known inside the local pass). */
+typedef enum { SPAVA_SCORE_LOGIT = 0, SPAVA_SCORE_PROB = 1 } spava_score_kind;
+
+/* Select the score kind (spava_score_kind) for this plan's later calls.  Host-side
+ * only; probability scores add an [hq][N] fp32 buffer to both workspaces, so query
+ * the workspace sizes after it.  Returns SPAVA_ERR_INVALID_ARG for a NULL plan or an
+ * unknown kind. */
+spava_status spava_plan_set_score_kind(spava_plan* plan, int32_t kind);
+
 /* Bytes of scratch the calls below need (scores, indices, passing K/V, text
  * partials, scheduler counters, error word).  0 if plan is NULL. */
 size_t spava_workspace_bytes(const spava_plan* plan);
@@ -273,7 +292,8 @@ spava_status spava_profile_end(spava_plan* plan);
 
 /* Name of a kernel label: 0 score, 1 select, 2 gather, 3 attention (prefill),
  * 4 lse merge, 5 attention (dense causal), 6 select + gather (fused, prefill),
- * 7 score-key fill/convert (two-stage), 8 attention stage 1, 9 attention stage 2. */
+ * 7 score-key fill/convert (two-stage), 8 attention stage 1, 9 attention stage 2,
+ * 10 probe-row lse (probability scores). */
 const char* spava_kernel_name(int32_t label);
 
 /* Static text of a status code. */

@@ -100,6 +100,18 @@ class Plan:
         self.workspace_bytes = int(self.lib.spava_workspace_bytes(self._h))
         self.two_stage_workspace_bytes = int(self.lib.spava_two_stage_workspace_bytes(self._h))
 
+    SCORE_KIND = {"logit": 0, "prob": 1}
+
+    def set_score_kind(self, kind: str) -> None:
+        """spava_plan_set_score_kind: "logit" (default) or "prob" (each probe row's
+        attention probability over its own block).  Call before new_workspace."""
+        if kind not in self.SCORE_KIND:
+            raise ValueError(f"score kind must be one of {sorted(self.SCORE_KIND)}")
+        _lib.check(self.lib.spava_plan_set_score_kind(self._h, self.SCORE_KIND[kind]), "spava_plan_set_score_kind")
+        self.score_kind = kind
+        self.workspace_bytes = int(self.lib.spava_workspace_bytes(self._h))
+        self.two_stage_workspace_bytes = int(self.lib.spava_two_stage_workspace_bytes(self._h))
+
     def set_debug(self, wait_limit_ns: int = 0, stall_producer: bool = False) -> None:
         _lib.check(self.lib.spava_plan_set_debug(self._h, int(wait_limit_ns), int(bool(stall_producer))),
                    "spava_plan_set_debug")

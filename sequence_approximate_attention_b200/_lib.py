@@ -40,6 +40,7 @@ SIGNATURES = {
     "spava_check_device_error": (c_int32, [c_void_p, c_void_p, c_void_p]),
     "spava_plan_set_debug": (c_int32, [c_void_p, ctypes.c_uint64, c_int32]),
     "spava_plan_set_score_reduce": (c_int32, [c_void_p, c_int32]),
+    "spava_plan_set_score_kind": (c_int32, [c_void_p, c_int32]),
     "spava_status_string": (ctypes.c_char_p, [c_int32]),
     "spava_last_error": (ctypes.c_char_p, []),
     "spava_last_launch_count": (c_int32, []),

@@ -48,6 +48,7 @@ enum : int {
   kOutTextPartial = 1,  // fp32 partial O and lse into text slot (out & 0xFFFF)
   kOutRowPartial = 2,   // fp32 partial O and lse of visual rows (local pass)
   kOutMerge = 3,        // lse-merge with the rows' partial, then bf16 O and lse
+  kOutLseOnly = 4,      // the rows' lse alone, into row_lse (probe rows of probability scores)
 };
 constexpr int kOutScore = 1 << 20;
 __host__ __device__ constexpr int make_out(int mode, int slot = 0, bool score = false) {
@@ -513,7 +514,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         const float2 r01 = fadd2(rs[0], rs[1]), r23 = fadd2(rs[2], rs[3]), r = fadd2(r01, r23);
         l_run = l_run * alpha + (r.x + r.y);
-        if (score_item && causal) {
+        if (score_item && causal && p.score_keys != nullptr) {
           // Two-stage flow: this item holds probe rows [aux - R, aux) of its host; fold
           // their raw q.k into the per-key scores (max over probe rows here, over the
           // group's query heads through the atomic max).  S is still intact in TMEM
@@ -615,6 +616,10 @@ __global__ void __launch_bounds__(384, 1)
         // fp32 partials: a text slot, or the visual rows of the local pass
         float* orow;
         float* lse_dst;
+        if (out_mode == kOutLseOnly) {
+          if (store) p.row_lse[static_cast<size_t>(it.q_head) * p.n_visual + grow] = lse_own;
+          continue;
+        }
         if (out_mode == kOutTextPartial) {
           const int slot = it.out & 0xFFFF, prow = grow - p.part_row0;
           orow = p.o_part + ((static_cast<size_t>(slot) * p.part_rows + prow) * p.hq + it.q_head) * D;

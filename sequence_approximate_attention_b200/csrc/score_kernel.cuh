@@ -3,6 +3,8 @@
 // local keys by query-to-context attention scores).
 //
 //   m_c(j)   = max over probe rows i in [e-R, e), i >= j, of (q_{i,c} . k_{j,g})
+//              (probability scores: of exp(scale q.k - lse_c(i)), lse_c(i) the probe
+//              row's log-sum-exp over the keys of its block it sees)
 //   score(g, j) = scale * reduce over the query heads c of group g of m_c(j),
 //   e = end of j's host block; reduce = max (default), sum or mean (the pages leave
 //   the combination open; max over heads and rows is the plainest reading), or none:
@@ -34,6 +36,10 @@ struct ScoreParams {
   int n_chunks;      // ceil(R / Rc)
   int head_reduce;   // 0 max, 1 sum, 2 mean over the group's query heads; 3 none (one
                      // score row per query head: scores is [hq][N])
+  // Probability scores: lse of every probe row over the keys of its block it sees,
+  // probe_lse[c * lse_stride + row] (query head c); nullptr for logit scores.
+  const float* probe_lse;
+  int lse_stride;
   int n_visual;      // N (row stride of scores)
   float scale;
   float* scores;     // [hkv][N]
@@ -267,6 +273,7 @@ __global__ void __launch_bounds__(256, 1)
       const int4 it = s_items[li];
       const int j = it.z + row;  // key position
       const int e = it.w;
+      const bool prob = p.probe_lse != nullptr;
       const bool by_head = p.head_reduce != 0;
       float mx_all = -INFINITY;   // max over heads and rows
       float mh[S::kMaxGroup];     // sum / mean: m_c(j) of each query head (indexed at run time)
@@ -282,7 +289,7 @@ __global__ void __launch_bounds__(256, 1)
         const int row0 = e - p.probe_r + c * Rc;         // first probe row of the chunk
         const int rc = min(Rc, p.probe_r - c * Rc);      // probe rows in it (a multiple of 16)
         const uint32_t ta = tl + b * 256;
-        if (!by_head && rc == Rc && it.z + 127 < row0) {
+        if (!by_head && !prob && rc == Rc && it.z + 127 < row0) {
           // Max over heads and rows with every column visible to every key of the
           // tile: order-free, whole 128-column TMEM loads and a three-input max tree.
           const int nc = Rc * G;
@@ -314,13 +321,26 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll 1
           for (int h = 0; h < G; ++h) {
             float m = -INFINITY;
+            const float* lse_h = prob ? p.probe_lse + static_cast<size_t>(it.y * G + h) * p.lse_stride + row0 : nullptr;
             for (int t0 = 0; t0 < rc; t0 += 16) {
               uint32_t v[16];
               tmem_ld_x16(ta + h * Rc + t0, v);
+              if (prob) {
+                // log probability scale * s - lse_c(row); lane t of each half-warp holds
+                // the lse of probe row row0 + t0 + t
+                const float lse_lane = __ldg(lse_h + t0 + (lane & 15));
 #pragma unroll
-              for (int t = 0; t < 16; ++t)
-                if (t0 + t >= t_min) m = fmaxf(m, __uint_as_float(v[t]));
+                for (int t = 0; t < 16; ++t) {
+                  const float lp = fmaf(__uint_as_float(v[t]), p.scale, -__shfl_sync(FULL, lse_lane, t));
+                  if (t0 + t >= t_min) m = fmaxf(m, lp);
+                }
+              } else {
+#pragma unroll
+                for (int t = 0; t < 16; ++t)
+                  if (t0 + t >= t_min) m = fmaxf(m, __uint_as_float(v[t]));
+              }
             }
+            if (prob) m = expf(m);
             if (by_head)
               mh[h] = fmaxf(mh[h], m);
             else
@@ -332,11 +352,12 @@ __global__ void __launch_bounds__(256, 1)
         if (lane == 0) mbar_arrive(acc_empty + b);
       }
       if (!ok) break;
+      const float out_scale = prob ? 1.0f : p.scale;  // probabilities carry the scale already
       if (p.head_reduce == 3) {
         if (j < e) {
 #pragma unroll 1
           for (int h = 0; h < G; ++h)
-            p.scores[(static_cast<size_t>(it.y) * G + h) * p.n_visual + j] = mh[h] * p.scale;
+            p.scores[(static_cast<size_t>(it.y) * G + h) * p.n_visual + j] = mh[h] * out_scale;
         }
         continue;
       }
@@ -347,7 +368,7 @@ __global__ void __launch_bounds__(256, 1)
         for (int h = 0; h < G; ++h) r += mh[h];
         if (p.head_reduce == 2) r = r / static_cast<float>(G);
       }
-      if (j < e) p.scores[static_cast<size_t>(it.y) * p.n_visual + j] = r * p.scale;
+      if (j < e) p.scores[static_cast<size_t>(it.y) * p.n_visual + j] = r * out_scale;
     }
   }
 

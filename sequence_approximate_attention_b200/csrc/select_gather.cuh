@@ -250,7 +250,12 @@ __global__ void __launch_bounds__(256) gather_passing_kernel(const uint4* __rest
 // Merge of split-KV partials through their lse (APB-V technical summary,
 // 2. System optimisations, "Fused context and query forward"):
 //   lse = log sum_k exp(lse_k),  O = sum_k exp(lse_k - lse) O_k.
-// One warp per (text row, head); slots with lse = -inf contribute nothing.
+// One warp per (text row, head); slots with lse = -inf contribute nothing.  Lane k
+// reads slot k's lse (so the slots' loads go out together), the maximum and the
+// weights are formed with shuffles, and the O partials are read kMergeUnroll slots
+// at a time.
+constexpr int kMergeUnroll = 4;
+
 __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict__ o_part,
                                                          const float* __restrict__ lse_part, int n_slots,
                                                          int part_rows, int hq, int d, int row0, int n_rows_out,
@@ -259,17 +264,42 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict_
   const int lane = lane_id();
   if (gw >= part_rows * hq) return;
   const int t = gw / hq, c = gw % hq;
+  // slot lse values, 32 per pass of the warp
   float m = -INFINITY;
-  for (int k = 0; k < n_slots; ++k) m = fmaxf(m, __ldg(lse_part + (static_cast<size_t>(k) * hq + c) * part_rows + t));
+  for (int k0 = 0; k0 < n_slots; k0 += 32) {
+    const int k = k0 + lane;
+    const float l = k < n_slots ? __ldg(lse_part + (static_cast<size_t>(k) * hq + c) * part_rows + t) : -INFINITY;
+    m = fmaxf(m, l);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
   float wsum = 0.f;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};  // d <= 128: lane owns d/32 <= 4 columns
   const int per = d / 32;
-  for (int k = 0; k < n_slots; ++k) {
-    const float l = __ldg(lse_part + (static_cast<size_t>(k) * hq + c) * part_rows + t);
-    const float w = (l == -INFINITY) ? 0.f : expf(l - m);
-    wsum += w;
-    const float* src = o_part + ((static_cast<size_t>(k) * part_rows + t) * hq + c) * d;
-    for (int e = 0; e < per; ++e) acc[e] += w * __ldg(src + lane + 32 * e);
+  for (int k0 = 0; k0 < n_slots; k0 += 32) {
+    const int kl = k0 + lane;
+    const float l = kl < n_slots ? __ldg(lse_part + (static_cast<size_t>(kl) * hq + c) * part_rows + t) : -INFINITY;
+    const float w_lane = (l == -INFINITY) ? 0.f : expf(l - m);
+    const int kn = min(32, n_slots - k0);
+    for (int kb = 0; kb < kn; kb += kMergeUnroll) {
+      float x[kMergeUnroll][4];
+#pragma unroll
+      for (int u = 0; u < kMergeUnroll; ++u) {
+        const int k = k0 + kb + u;
+        const float* src = o_part + ((static_cast<size_t>(min(k, n_slots - 1)) * part_rows + t) * hq + c) * d;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[u][e] = (e < per && kb + u < kn) ? __ldg(src + lane + 32 * e) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kMergeUnroll; ++u) {
+        const float w = __shfl_sync(0xffffffffu, w_lane, (kb + u) & 31);
+        if (kb + u < kn) {
+          wsum += w;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[e] = fmaf(w, x[u][e], acc[e]);
+        }
+      }
+    }
   }
   const float inv = 1.0f / wsum;
   __nv_bfloat16* dst = o + (static_cast<size_t>(row0 + t) * hq + c) * d;

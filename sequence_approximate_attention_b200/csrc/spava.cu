@@ -102,6 +102,7 @@ struct spava_plan {
   // score chunking: Rc probe tokens per MMA N chunk
   int rc = 0, n_chunks = 0;
   int score_reduce = SPAVA_SCORE_MAX;  // spava_plan_set_score_reduce
+  int score_kind = SPAVA_SCORE_LOGIT;  // spava_plan_set_score_kind
   // device table (owned)
   void* dtab = nullptr;
   int* d_off = nullptr;
@@ -113,6 +114,8 @@ struct spava_plan {
   int n_items_local = 0;
   AttnItem* d_items_remote = nullptr;  // two-stage flow, second launch
   int n_items_remote = 0;
+  AttnItem* d_items_probe = nullptr;   // probability scores: lse of every host's probe rows
+  int n_items_probe = 0;
   int4* d_score_pre = nullptr;  // hosts 0..H-2
   int n_score_pre = 0;
   int4* d_score_all = nullptr;  // all hosts
@@ -120,6 +123,7 @@ struct spava_plan {
   // workspace layout
   size_t ws_err = 0, ws_scores = 0, ws_idx = 0, ws_kp = 0, ws_vp = 0, ws_opart = 0, ws_lpart = 0, ws_total = 0;
   size_t ws_row_o = 0, ws_row_lse = 0, ws_qkeys = 0, ws_total_two_stage = 0;  // two-stage flow only
+  size_t ws_probe_lse = 0;  // probability scores: [hq][N] lse (probe rows only)
   // debug knobs
   uint64_t wait_limit_ns = spava::kDefaultWaitLimitNs;
   int stall_producer = 0;
@@ -136,7 +140,7 @@ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 enum KernelLabel {
   kLabScore = 0, kLabSelect = 1, kLabGather = 2, kLabAttn = 3, kLabMerge = 4, kLabDense = 5, kLabSelectGather = 6,
-  kLabFill = 7, kLabAttnLocal = 8, kLabAttnRemote = 9
+  kLabFill = 7, kLabAttnLocal = 8, kLabAttnRemote = 9, kLabProbeLse = 10
 };
 
 void mark(const spava_plan* p, int label, cudaStream_t st) {
@@ -288,6 +292,28 @@ std::vector<AttnItem> build_remote_items(const spava_plan& p) {
   return v;
 }
 
+// Probability scores: the last R rows of every host over its own block (causal), lse
+// only -- each probe row's log-sum-exp over the keys of its block it sees.
+std::vector<AttnItem> build_probe_items(const spava_plan& p) {
+  std::vector<AttnItem> v;
+  std::vector<int> group;
+  if (p.R == 0) return v;
+  for (int h = 0; h < p.H; ++h) {
+    const int a = p.off[h], e = p.off[h + 1];
+    for (int r0 = e - p.R; r0 < e; r0 += 256) {
+      const int rows = std::min(256, e - r0);
+      for (int c = 0; c < p.hq; ++c) {
+        AttnItem it = blank_item(r0, rows, c, spava::make_out(spava::kOutLseOnly));
+        it.seg[0] = AttnSeg{a, r0 + rows - a, spava::kSegCausal, 0};
+        v.push_back(it);
+        group.push_back(h);
+      }
+    }
+  }
+  sort_host_major(v, group, p.hq / p.hkv);
+  return v;
+}
+
 std::vector<AttnItem> build_dense_items(const spava_plan& p) {
   std::vector<AttnItem> v;
   const int NT = p.N + p.T;
@@ -342,6 +368,8 @@ void layout_workspace(spava_plan* p) {
   o = align_up(o + hm1 * rows * P * d * 2, 256);
   p->ws_vp = o;
   o = align_up(o + hm1 * rows * P * d * 2, 256);
+  p->ws_probe_lse = o;
+  if (p->score_kind == SPAVA_SCORE_PROB) o = align_up(o + hq * n_visual * 4, 256);
   p->ws_opart = o;
   o = align_up(o + static_cast<size_t>(p->H + 1) * n_text * hq * d * 4, 256);
   p->ws_lpart = o;
@@ -382,6 +410,10 @@ spava_status launch_score(const spava_plan* p, const void* q, const void* k, flo
   sp.chunk_tokens = p->rc;
   sp.n_chunks = p->n_chunks;
   sp.head_reduce = p->score_reduce;
+  sp.probe_lse = p->score_kind == SPAVA_SCORE_PROB
+                     ? reinterpret_cast<const float*>(static_cast<const uint8_t*>(ws) + p->ws_probe_lse)
+                     : nullptr;
+  sp.lse_stride = p->N;
   sp.n_visual = p->N;
   sp.scale = p->scale;
   sp.scores = scores;
@@ -509,11 +541,25 @@ spava_status launch_attn(const spava_plan* p, const AttnItem* items, int n_items
   const int grid = std::min(n_items, p->num_sms);
   mark(p, items == p->d_items_dense ? kLabDense
              : items == p->d_items_local ? kLabAttnLocal
-             : items == p->d_items_remote ? kLabAttnRemote : kLabAttn, st);
+             : items == p->d_items_remote ? kLabAttnRemote
+             : items == p->d_items_probe ? kLabProbeLse : kLabAttn, st);
   spava::attn_fwd_kernel<D><<<grid, S::kThreads, S::kSmemBytes, st>>>(tmQ, tmK, tmV, tmKp, tmVp, ap);
   SPAVA_CUDA(cudaGetLastError());
   ++g_last_launches;
   return SPAVA_OK;
+}
+
+// Probability scores: the lse of every host's probe rows over its block, into the
+// workspace (the items' O is not stored; V only has to be a readable K/V tensor).
+spava_status launch_probe_lse(const spava_plan* p, const void* q, const void* k, const void* v, void* ws,
+                              cudaStream_t st) {
+  if (p->score_kind != SPAVA_SCORE_PROB) return SPAVA_OK;
+  TwoStageBufs t;
+  t.row_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + p->ws_probe_lse);
+  return p->d == 128 ? launch_attn<128>(p, p->d_items_probe, p->n_items_probe, q, k, v, nullptr, nullptr, nullptr,
+                                        nullptr, ws, st, t)
+                     : launch_attn<64>(p, p->d_items_probe, p->n_items_probe, q, k, v, nullptr, nullptr, nullptr,
+                                       nullptr, ws, st, t);
 }
 
 spava_status launch_merge(const spava_plan* p, void* o, float* lse, void* ws, cudaStream_t st) {
@@ -635,12 +681,14 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   const auto dense = build_dense_items(*p);
   const auto local = build_local_items(*p);
   const auto remote = build_remote_items(*p);
+  const auto probe = build_probe_items(*p);
   const auto sc_pre = build_score_items(*p, n_hosts - 1);
   const auto sc_all = build_score_items(*p, n_hosts);
   p->n_items_pre = static_cast<int>(pre.size());
   p->n_items_dense = static_cast<int>(dense.size());
   p->n_items_local = static_cast<int>(local.size());
   p->n_items_remote = static_cast<int>(remote.size());
+  p->n_items_probe = static_cast<int>(probe.size());
   p->n_score_pre = static_cast<int>(sc_pre.size());
   p->n_score_all = static_cast<int>(sc_all.size());
   // One device table, each array 256-byte aligned.
@@ -658,6 +706,7 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   const size_t o_sall = put(sc_all.data(), sc_all.size() * sizeof(int4));
   const size_t o_local = put(local.data(), local.size() * sizeof(AttnItem));
   const size_t o_remote = put(remote.data(), remote.size() * sizeof(AttnItem));
+  const size_t o_probe = put(probe.data(), probe.size() * sizeof(AttnItem));
   e = cudaMalloc(&p->dtab, host.size());
   if (e != cudaSuccess) return bail(fail(SPAVA_ERR_CUDA, "cudaMalloc(plan table): %s", cudaGetErrorString(e)));
   e = cudaMemcpy(p->dtab, host.data(), host.size(), cudaMemcpyHostToDevice);
@@ -670,6 +719,7 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   p->d_score_all = reinterpret_cast<int4*>(base + o_sall);
   p->d_items_local = reinterpret_cast<AttnItem*>(base + o_local);
   p->d_items_remote = reinterpret_cast<AttnItem*>(base + o_remote);
+  p->d_items_probe = reinterpret_cast<AttnItem*>(base + o_probe);
   *out = p;
   return ok();
 }
@@ -706,6 +756,15 @@ spava_status spava_plan_set_score_reduce(spava_plan* p, int32_t mode) {
   return ok();
 }
 
+spava_status spava_plan_set_score_kind(spava_plan* p, int32_t kind) {
+  if (!p) return fail(SPAVA_ERR_INVALID_ARG, "plan is NULL");
+  if (kind != SPAVA_SCORE_LOGIT && kind != SPAVA_SCORE_PROB)
+    return fail(SPAVA_ERR_INVALID_ARG, "unknown score kind %d", kind);
+  p->score_kind = kind;
+  layout_workspace(p);  // probability scores keep the probe rows' lse in the workspace
+  return ok();
+}
+
 spava_status spava_plan_set_debug(spava_plan* p, uint64_t wait_limit_ns, int32_t stall_producer) {
   if (!p) return fail(SPAVA_ERR_INVALID_ARG, "plan is NULL");
   p->wait_limit_ns = wait_limit_ns ? wait_limit_ns : spava::kDefaultWaitLimitNs;
@@ -726,6 +785,7 @@ spava_status spava_score_select(const spava_plan* p, const void* q, const void* 
   if ((s = begin_call(p, ws, st)) != SPAVA_OK) return s;
   if (!(flags & SPAVA_SCORES_GIVEN) && p->H >= 1) {
     if (p->R == 0) return fail(SPAVA_ERR_INVALID_ARG, "plan has R = 0: nothing to score");
+    if ((s = launch_probe_lse(p, q, k, k, ws, st)) != SPAVA_OK) return s;
     s = p->d == 128 ? launch_score<128>(p, q, k, scores, true, ws, st) : launch_score<64>(p, q, k, scores, true, ws, st);
     if (s != SPAVA_OK) return s;
   }
@@ -763,6 +823,7 @@ spava_status spava_attn_prefill(const spava_plan* p, const void* q, const void* 
   void* kp = w + p->ws_kp;
   void* vp = w + p->ws_vp;
   if (p->H >= 2 && p->P > 0) {
+    if ((s = launch_probe_lse(p, q, k, v, ws, st)) != SPAVA_OK) return s;
     s = p->d == 128 ? launch_score<128>(p, q, k, scores, false, ws, st) : launch_score<64>(p, q, k, scores, false, ws, st);
     if (s != SPAVA_OK) return s;
     if ((s = launch_select(p, scores, idx, st, k, v, kp, vp)) != SPAVA_OK) return s;
@@ -846,11 +907,20 @@ spava_status spava_attn_prefill_two_stage(const spava_plan* p, const void* q, co
   ts.row_lse = reinterpret_cast<float*>(w + p->ws_row_lse);
   // Max over heads: one key row per KV head, turned into scores in place.  Sum / mean:
   // one key row per query head, combined into the scores after the local pass.
+  // Probability scores need each probe row's final lse: scored by the score kernel
+  // instead of being folded into the local pass.
+  const bool prob = p->score_kind == SPAVA_SCORE_PROB;
   ts.per_qhead = p->score_reduce != SPAVA_SCORE_MAX;
-  ts.score_keys = ts.per_qhead ? reinterpret_cast<unsigned int*>(w + p->ws_qkeys) : reinterpret_cast<unsigned int*>(scores);
+  ts.score_keys = prob ? nullptr
+                  : ts.per_qhead ? reinterpret_cast<unsigned int*>(w + p->ws_qkeys)
+                                 : reinterpret_cast<unsigned int*>(scores);
   const size_t n_keys = static_cast<size_t>(ts.per_qhead ? p->hq : p->hkv) * p->N;
   const int grid_small = std::max(1, std::min(p->num_sms * 4, static_cast<int>((n_keys + 255) / 256)));
-  if (scores_needed(*p)) {
+  if (scores_needed(*p) && prob) {
+    if ((s = launch_probe_lse(p, q, k, v, ws, st)) != SPAVA_OK) return s;
+    s = p->d == 128 ? launch_score<128>(p, q, k, scores, false, ws, st) : launch_score<64>(p, q, k, scores, false, ws, st);
+    if (s != SPAVA_OK) return s;
+  } else if (scores_needed(*p)) {
     mark(p, kLabFill, st);
     spava::fill_u32_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, n_keys, spava::kOrderedNegInf);
     SPAVA_CUDA(cudaGetLastError());
@@ -861,17 +931,19 @@ spava_status spava_attn_prefill_two_stage(const spava_plan* p, const void* q, co
                   : launch_attn<64>(p, p->d_items_local, p->n_items_local, q, k, v, nullptr, nullptr, o, lse, ws, st, ts);
   if (s != SPAVA_OK) return s;
   if (scores_needed(*p)) {
-    mark(p, kLabFill, st);
-    if (p->score_reduce == SPAVA_SCORE_PER_QUERY_HEAD)  // one score row per query head: convert
-      spava::combine_head_keys_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, scores, p->hq, 1,
-                                                                   static_cast<size_t>(p->N), SPAVA_SCORE_SUM);
-    else if (ts.per_qhead)
-      spava::combine_head_keys_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, scores, p->hkv, p->hq / p->hkv,
-                                                                   static_cast<size_t>(p->N), p->score_reduce);
-    else
-      spava::keys_to_scores_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, n_keys);
-    SPAVA_CUDA(cudaGetLastError());
-    ++g_last_launches;
+    if (!prob) {
+      mark(p, kLabFill, st);
+      if (p->score_reduce == SPAVA_SCORE_PER_QUERY_HEAD)  // one score row per query head: convert
+        spava::combine_head_keys_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, scores, p->hq, 1,
+                                                                     static_cast<size_t>(p->N), SPAVA_SCORE_SUM);
+      else if (ts.per_qhead)
+        spava::combine_head_keys_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, scores, p->hkv, p->hq / p->hkv,
+                                                                     static_cast<size_t>(p->N), p->score_reduce);
+      else
+        spava::keys_to_scores_kernel<<<grid_small, 256, 0, st>>>(ts.score_keys, n_keys);
+      SPAVA_CUDA(cudaGetLastError());
+      ++g_last_launches;
+    }
     if ((s = launch_select(p, scores, idx, st, k, v, kp, vp)) != SPAVA_OK) return s;
   }
   // stage 2: remote pass over [anchor | passing], lse-merged with the local partials
@@ -950,6 +1022,7 @@ const char* spava_kernel_name(int32_t label) {
     case kLabFill: return "score_keys";
     case kLabAttnLocal: return "attention_local";
     case kLabAttnRemote: return "attention_remote";
+    case kLabProbeLse: return "probe_lse";
   }
   return "unknown";
 }
