@@ -56,6 +56,18 @@ def dense_pairs(cfg):
     return n * (n + 1) // 2
 
 
+def score_flops(cfg, sizes):
+    """Tensor-core work of the score kernel: every scored key meets the R probe rows of
+    each of the G query heads of its group (2 d FLOP each); the N chunks are Rc G
+    columns wide, so a short last chunk still costs its full width."""
+    d, hq, hkv, H, R = cfg.head_dim, cfg.hq, cfg.hkv, cfg.n_hosts, cfg.probe_r
+    G = hq // hkv
+    n_scored = int(sum(int(b) for b in sizes[:H - 1]))
+    rc = min(max(16, 16 * (256 // (16 * G))), R)
+    cols = -(-R // rc) * rc * G
+    return 2.0 * d * cols * n_scored * hkv
+
+
 def select_gather_bytes(cfg, sizes):
     """Algorithmic HBM bytes of the score, select and gather kernels of one step."""
     d, hq, hkv, H, P, R, N = cfg.head_dim, cfg.hq, cfg.hkv, cfg.n_hosts, cfg.passing, cfg.probe_r, cfg.n_visual
@@ -394,6 +406,12 @@ def main():
         if name in avg:
             gbs = sgb[name] / (avg[name] / 1e3) / 1e9
             hbm[name] = {"ms": avg[name], "bytes": sgb[name], "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]}
+    if "score" in hbm:
+        # the score kernel sits at its ridge point: report the tensor side too
+        sf = score_flops(cfg, sizes)
+        hbm["score"]["flops"] = sf
+        hbm["score"]["TFLOP/s"] = sf / (avg["score"] / 1e3) / 1e12
+        hbm["score"]["frac_of_tensor_peak"] = hbm["score"]["TFLOP/s"] / peaks["bf16_tflops"]
     ssg_names = [n for n in ("score", "select", "gather", "select_gather") if n in avg]
     ssg_ms = sum(avg[n] for n in ssg_names)
     ssg_bytes = sum(sgb[n] for n in ssg_names)
