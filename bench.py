@@ -312,6 +312,9 @@ def main():
                     help="single: one attention pass per host (default); two_stage: local pass with fused "
                          "probe scores, then the remote pass merged through the lse")
     ap.add_argument("--e2e-steps", type=int, default=8)
+    ap.add_argument("--ttft-layers", type=int, default=0,
+                    help="also time a synthetic prefill of this many attention blocks (projections + attention), "
+                         "approximate vs dense")
     ap.add_argument("--dense", type=int, default=1, help="also time the dense causal kernel (0/1)")
     ap.add_argument("--cpu-baseline", type=int, default=1)
     ap.add_argument("--cpu-rows", type=int, default=1024)
@@ -494,6 +497,32 @@ def main():
                "serial_value": job_throughput(world, NT, max(2, args.e2e_steps // 2), ts)}
         del pipe
 
+    # time-to-first-token style: L attention blocks (random weights, plain GEMM
+    # projections around the library's attention), approximate vs dense attention
+    ttft = None
+    if args.ttft_layers > 0:
+        from sequence_approximate_attention_b200.layer_stack import LayerStack
+        hidden = cfg.hq * cfg.head_dim
+        stack = LayerStack(plan, hidden, args.ttft_layers, seed=cfg.seed, two_stage=two_stage)
+        x0 = (torch.randn(NT, hidden, generator=torch.Generator().manual_seed(cfg.seed)) * 0.5).to(torch.bfloat16).to(dev)
+        times = {}
+        for dense_mode in (False, True):
+            stack.forward(x0, dense=dense_mode)
+            torch.cuda.synchronize(dev)
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(2):
+                stack.forward(x0, dense=dense_mode)
+            t1.record(stream)
+            torch.cuda.synchronize(dev)
+            times["dense" if dense_mode else "approx"] = max_over_ranks(t0.elapsed_time(t1), dev) / 2
+        ttft = {"layers": args.ttft_layers, "hidden": hidden, "tokens": NT, "approx_ms": times["approx"],
+                "dense_ms": times["dense"], "speedup": times["dense"] / times["approx"],
+                "projection_tflop_per_layer": stack.flops()["projections"] / 1e12,
+                "note": "attention blocks only (RMSNorm, QKV and output projections, attention, residual); "
+                        "random weights, no rotary embedding, no MLP"}
+        del stack
+
     cpu = None
     if args.cpu_baseline and rank == 0 and world == 1:
         t_full, desc, work = oracle_sample(cfg, g, 7, rows=args.cpu_rows)
@@ -507,7 +536,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "b200", "flow": args.flow,
             "config": workload_config(cfg),
             "tflops_step": step_tflops, "tflops_step_frac": step_tflops / peaks["bf16_tflops"],
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "ttft": ttft,
             "clocks": clk, "dense_causal": dense,
         }
         print(json.dumps(line), flush=True)
