@@ -193,3 +193,58 @@ def test_fullsize_two_stage_flow(fullsize_run):
     assert do <= O_TOL and dl <= LSE_TOL, (cfg.name, do, dl)
     del ws
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("reduce,kind", [("per_query_head", "logit"), ("max", "prob")])
+def test_fullsize_score_variants_qwen64k(reduce, kind):
+    """The score variants at full size (qwen64k, 28/4 heads): per-query-head selection
+    (scores, indices and passing buffers per query head) and probability scores (probe
+    rows' lse by the attention kernel, then the score kernel).  Every score of hosts
+    0..H-2 against the fp64 oracle (probabilities in the log domain), selection
+    bit-exact on the GPU's own scores, sampled outputs against the oracle re-run with
+    the GPU's indices."""
+    cfg = CONFIGS["qwen64k"]
+    g = generate(cfg)
+    sizes = [int(x) for x in g["host_sizes"]]
+    dev = {x: to_device_bf16(g[x]) for x in ("q", "k", "v")}
+    plan = sab.Plan(cfg.n_visual, cfg.n_text, cfg.n_hosts, sizes, cfg.anchor, cfg.passing, cfg.probe_r,
+                    cfg.hq, cfg.hkv, cfg.head_dim)
+    plan.set_score_reduce(reduce)
+    plan.set_score_kind(kind)
+    ws = plan.new_workspace()
+    scores = torch.empty(plan.scores_shape(), dtype=torch.float32, device="cuda")
+    idx = torch.empty(plan.idx_shape(), dtype=torch.int32, device="cuda")
+    o, lse = sab.attn_prefill(plan, dev["q"], dev["k"], dev["v"], scores_out=scores, idx_out=idx, workspace=ws)
+    sab.check_device_error(plan, ws)
+    off = orc.host_offsets(sizes)
+    q, k, v = (LazyF64(g[x]) for x in ("q", "k", "v"))
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    G = cfg.hq // cfg.hkv
+    sc = scores.cpu().numpy()
+    for h in range(cfg.n_hosts - 1):
+        a, e = int(off[h]), int(off[h + 1])
+        sub = orc.host_offsets([e - a])
+        qh, kh = q[a:e], k[a:e]
+        ref = orc.probe_scores(qh, kh, sub, cfg.probe_r, scale, "none" if reduce == "per_query_head" else reduce, kind)
+        _, tol = _score_tolerance_and_ref(qh, kh, sub, cfg.probe_r, scale, [0])
+        t = np.stack([tol[(0, gg)] for gg in range(cfg.hkv)])
+        if reduce == "per_query_head":
+            t = np.repeat(t, G, axis=0)
+        got = sc[:, a:e].astype(np.float64)
+        if kind == "prob":
+            err = np.abs(np.log(got) - np.log(ref))
+            assert (err <= t + 5e-4).all(), (h, float(err.max()))
+        else:
+            assert (np.abs(got - ref) <= t).all(), (h, float(np.abs(got - ref).max()))
+    sel = idx.cpu().numpy().astype(np.int64)
+    np.testing.assert_array_equal(sel, orc.select_passing(sc, off, cfg.anchor, cfg.passing))
+    rng = np.random.default_rng(cfg.seed + 2)
+    rows, heads = _sample_rows(cfg, off, rng, n_random=24)
+    O_ref, L_ref = orc.attention_rows(q, k, v, off, cfg.anchor, sel, scale, rows, heads)
+    rt, ht = torch.tensor(rows, device="cuda"), torch.tensor(heads, device="cuda")
+    do = np.abs(o[rt, ht].float().cpu().numpy() - O_ref).max()
+    dl = np.abs(lse[ht, rt].cpu().numpy() - L_ref).max()
+    assert do <= O_TOL and dl <= LSE_TOL, (reduce, kind, do, dl)
+    plan.close()
+    del dev, o, lse, ws
+    torch.cuda.empty_cache()
