@@ -181,18 +181,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Per-warpgroup register budget (all four warps of a warpgroup execute the same
-// call).  The budgets of all warpgroups must add up to at most the registers the
-// CTA was launched with, or the increase waits forever.
-template <uint32_t kRegs>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
-template <uint32_t kRegs>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
-
 // Order-preserving map fp32 -> uint32 (larger float -> larger key).  -0.0 is first
 // made +0.0, so both zeros get the same key.  NaN never reaches here (scores of
 // finite bf16 inputs are finite).
