@@ -122,3 +122,31 @@ def test_gather_per_query_head(name):
             assert torch.equal(kp16[c, h], k16[rows, c // G]), (name, c, h)
             assert torch.equal(vp16[c, h], v16[rows, c // G]), (name, c, h)
     plan.close()
+
+
+@pytest.mark.parametrize("sizes,anchor,passing", [([8192] * 3, 1024, 1024), ([300, 500, 224], 10, 290),
+                                                  ([1000, 24], 0, 1)])
+def test_per_query_head_select_bit_exact_with_ties(sizes, anchor, passing):
+    """Selection rows per query head (hq = 8 rows of scores) through the given-scores
+    path, on adversarial scores (exact ties, +-0, huge values, a near-equal ramp):
+    bit-exact against the oracle's selection of the same fp32 scores."""
+    rng = np.random.default_rng(len(sizes) * 7 + passing)
+    hq, hkv = 8, 2
+    N = int(sum(sizes))
+    cfg = TINY.with_(n_visual=N, n_hosts=len(sizes), anchor=anchor, passing=passing, probe_r=16,
+                     hq=hq, hkv=hkv, head_dim=64)
+    plan = make_plan(sab, cfg, sizes)
+    plan.set_score_reduce("per_query_head")
+    s = rng.integers(-4, 5, size=(hq, N)).astype(np.float32)
+    s[0, ::7] = -0.0
+    s[0, 3::7] = 0.0
+    s[1] = 2.5
+    s[2] = rng.standard_normal(N).astype(np.float32) * np.float32(1e30)
+    s[3] = np.float32(1.0) + np.arange(N, dtype=np.float32) * np.float32(1e-7)
+    scores = torch.from_numpy(s).cuda()
+    _, idx = sab.score_select(plan, None, None, scores=scores, scores_given=True)
+    torch.cuda.synchronize()
+    off = orc.host_offsets(sizes)
+    assert idx.shape == (len(sizes) - 1, hq, passing)
+    np.testing.assert_array_equal(idx.cpu().numpy(), orc.select_passing(s, off, anchor, passing))
+    plan.close()
