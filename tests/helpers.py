@@ -78,3 +78,20 @@ def compare_attention(o_gpu, lse_gpu, O_ref, L_ref, what=""):
 
 def default_scale(cfg):
     return 1.0 / math.sqrt(cfg.head_dim)
+
+
+def adversarial_scores(rng, rows, N):
+    """fp32 scores [rows, N] built to break a selection: heavy exact ties, +-0, one row
+    all equal, values near the fp32 limits, and a ramp whose steps are one or two ulps."""
+    s = rng.integers(-4, 5, size=(rows, N)).astype(np.float32)   # heavy exact ties
+    s[0, ::7] = -0.0
+    s[0, 3::7] = 0.0
+    if rows > 1:
+        s[1] = 2.5                                               # all equal
+    if rows > 2:
+        s[2] = rng.standard_normal(N).astype(np.float32) * np.float32(1e30)
+        s[2, 100:110] = np.float32(3.0e38)
+        s[2, 200:210] = np.float32(-3.0e38)
+    if rows > 3:
+        s[3] = np.float32(1.0) + np.arange(N, dtype=np.float32) * np.float32(1e-7)  # near-equal ramp
+    return s

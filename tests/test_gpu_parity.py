@@ -18,8 +18,8 @@ import torch
 from oracle import spava_oracle as orc
 from workloads import CONFIGS, generate
 
-from .helpers import (check_selection_vs_fp64, compare_attention, inputs, make_plan, score_tolerance,
-                      to_device_bf16)
+from .helpers import (adversarial_scores, check_selection_vs_fp64, compare_attention, inputs, make_plan,
+                      score_tolerance, to_device_bf16)
 
 pytestmark = pytest.mark.gpu
 
@@ -130,21 +130,6 @@ def test_score_select_all_hosts(name):
     plan.close()
 
 
-def _adversarial_scores(rng, hkv, N):
-    s = rng.integers(-4, 5, size=(hkv, N)).astype(np.float32)   # heavy exact ties
-    s[0, ::7] = -0.0
-    s[0, 3::7] = 0.0
-    if hkv > 1:
-        s[1] = 2.5                                               # all equal
-    if hkv > 2:
-        s[2] = rng.standard_normal(N).astype(np.float32) * np.float32(1e30)
-        s[2, 100:110] = np.float32(3.0e38)
-        s[2, 200:210] = np.float32(-3.0e38)
-    if hkv > 3:
-        s[3] = np.float32(1.0) + np.arange(N, dtype=np.float32) * np.float32(1e-7)  # near-equal ramp
-    return s
-
-
 @pytest.mark.parametrize("sizes,anchor,passing", [
     ([8192] * 3, 1024, 1024), ([4096, 12288, 6144, 9216], 2048, 2048), ([300, 500, 224], 10, 290),
     ([64, 64], 0, 64), ([1000, 24], 0, 1)])
@@ -155,7 +140,7 @@ def test_select_bit_exact_with_ties(sizes, anchor, passing):
     cfg = TINY.with_(n_visual=N, n_hosts=len(sizes), anchor=anchor, passing=passing, probe_r=16,
                      hq=4, hkv=hkv, head_dim=64)
     plan = make_plan(sab, cfg, sizes)
-    s = _adversarial_scores(rng, hkv, N)
+    s = adversarial_scores(rng, hkv, N)
     scores = torch.from_numpy(s).cuda()
     _, idx = sab.score_select(plan, None, None, scores=scores, scores_given=True)
     torch.cuda.synchronize()

@@ -20,7 +20,7 @@ import torch
 from oracle import spava_oracle as orc
 from workloads import CONFIGS
 
-from .helpers import check_selection_vs_fp64, compare_attention, inputs, make_plan, score_tolerance
+from .helpers import adversarial_scores, check_selection_vs_fp64, compare_attention, inputs, make_plan, score_tolerance
 
 pytestmark = pytest.mark.gpu
 
@@ -137,12 +137,7 @@ def test_per_query_head_select_bit_exact_with_ties(sizes, anchor, passing):
                      hq=hq, hkv=hkv, head_dim=64)
     plan = make_plan(sab, cfg, sizes)
     plan.set_score_reduce("per_query_head")
-    s = rng.integers(-4, 5, size=(hq, N)).astype(np.float32)
-    s[0, ::7] = -0.0
-    s[0, 3::7] = 0.0
-    s[1] = 2.5
-    s[2] = rng.standard_normal(N).astype(np.float32) * np.float32(1e30)
-    s[3] = np.float32(1.0) + np.arange(N, dtype=np.float32) * np.float32(1e-7)
+    s = adversarial_scores(rng, hq, N)
     scores = torch.from_numpy(s).cuda()
     _, idx = sab.score_select(plan, None, None, scores=scores, scores_given=True)
     torch.cuda.synchronize()
