@@ -267,6 +267,97 @@ size_t spava_two_stage_workspace_bytes(const spava_plan* plan);
 spava_status spava_dense_causal(const spava_plan* plan, const void* q, const void* k,
                                 const void* v, void* o, float* lse, void* ws, void* stream);
 
+/*
+ * Sharded prefill: the host blocks spread over `world` ranks, one process per GPU,
+ * each rank running the work of its own hosts (APB-V technical summary, 1. Framework
+ * design, "Context splitting & ZigZag arrangement": a physical host runs a pair of
+ * virtual hosts; 2. System optimisations, "Overlapped communication": passing blocks
+ * and partial query results travel while attention runs).  The library computes; the
+ * caller moves bytes between the ranks between the stages (an all-gather of each
+ * exchange buffer, a broadcast of the anchor rows), on a stream of its own so that
+ * the transfers overlap the next stage.
+ *
+ * Ownership policies (spava_shard_owners):
+ *   SPAVA_SHARD_CONTIGUOUS  rank r runs hosts [r*H/world, (r+1)*H/world).
+ *   SPAVA_SHARD_ZIGZAG      the hosts form rounds of 2*world; in each round rank r runs
+ *                           hosts r and 2*world-1-r (a later host attends to more
+ *                           passing rows, so the pairs carry equal passing lengths).
+ */
+typedef enum { SPAVA_SHARD_CONTIGUOUS = 0, SPAVA_SHARD_ZIGZAG = 1 } spava_shard_policy;
+
+/* Host-side only (no device needed): owner_out[h] = the rank that runs host h, for a
+ * HOST array of n_hosts ints.  CONTIGUOUS needs n_hosts % world == 0, ZIGZAG
+ * n_hosts % (2 * world) == 0; otherwise, or for a NULL array or world < 1, returns
+ * SPAVA_ERR_INVALID_ARG and writes nothing. */
+spava_status spava_shard_owners(int32_t n_hosts, int32_t world, int32_t policy, int32_t* owner_out);
+
+/* Make `plan` run rank `rank` of `world`, host h on rank owner[h] (HOST array of H
+ * ints in [0, world), copied; every rank of a job passes the same array).  Builds this
+ * rank's work lists into a device table owned by the plan (synchronises the device
+ * when it replaces an earlier one) and sizes the sharded workspace; query the layout
+ * afterwards, and again after spava_plan_set_score_reduce / _kind.  Returns
+ * SPAVA_ERR_INVALID_ARG for a bad rank, world or owner entry. */
+spava_status spava_plan_set_shard(spava_plan* plan, int32_t rank, int32_t world, const int32_t* owner);
+
+/* Workspace layout of the sharded prefill (byte offsets into the workspace).
+ *   pass_k / pass_v   passing exchange buffers, bf16 [world][pass_slots][P][rows][d]
+ *                     (rows = selection rows): slot s of rank r holds the passing rows
+ *                     of rank r's s-th own host < H-1 (ascending), row j of selection
+ *                     row g at [r][s][j][g].  Rank r's part is the contiguous run
+ *                     [r * pass_bytes_per_rank, (r+1) * pass_bytes_per_rank).
+ *   text_o / text_lse text partial exchange buffers, fp32 [world][text_slots][T][hq][d]
+ *                     and [world][text_slots][hq][T]: slot s of rank r is its s-th text
+ *                     piece (the text rows over each own host's block, ascending, then
+ *                     on the owner of host H-1 the text rows' own causal part); unused
+ *                     slots hold O = 0, lse = -inf.  Parts per rank as above.
+ *   scores, idx       this rank's scores [rows][N] and selection [H-1][rows][P] (the
+ *                     entries of its own hosts < H-1 are written).
+ */
+typedef struct {
+  uint64_t workspace_bytes;
+  uint64_t pass_k_offset, pass_v_offset, pass_bytes_per_rank;
+  uint64_t text_o_offset, text_o_bytes_per_rank;
+  uint64_t text_lse_offset, text_lse_bytes_per_rank;
+  uint64_t scores_offset, idx_offset;
+  int32_t pass_slots, text_slots;
+} spava_shard_layout;
+
+/* Fill *out for a plan after spava_plan_set_shard; SPAVA_ERR_INVALID_ARG otherwise. */
+spava_status spava_shard_query(const spava_plan* plan, spava_shard_layout* out);
+
+/* Stages of the sharded prefill, run in this order on every rank:
+ *   SPAVA_SHARD_SELECT  score the own hosts < H-1 (score kernel), select their top P
+ *                       and write the passing rows into this rank's part of pass_k /
+ *                       pass_v.  Reads the probe rows of q and the own blocks of k, v.
+ *                       Clears the workspace error word.
+ *     caller: all-gather pass_k and pass_v; broadcast k, v rows [0, A) from the owner
+ *     of host 0 into every rank's k, v (both may overlap LOCAL).
+ *   SPAVA_SHARD_LOCAL   own hosts' rows over their own block (causal): final O/lse for
+ *                       hosts without a remote part (host 0), fp32 row partials for the
+ *                       others; the text rows over each own block into this rank's
+ *                       text slots.  Reads own rows of q, k, v and the text rows of q
+ *                       (and of k, v on the owner of host H-1).
+ *     caller: all-gather text_o and text_lse (may overlap REMOTE).
+ *   SPAVA_SHARD_REMOTE  own hosts h >= 1 over [anchor | passing of hosts < h], merged
+ *                       with their row partials into the final O/lse of their rows.
+ *                       Needs the gathered pass_k / pass_v and the anchor rows.
+ *   SPAVA_SHARD_MERGE   text rows from all ranks' text slots (needs the gathered
+ *                       text_o / text_lse): final O/lse of rows [N, N+T).
+ * q, k, v, o [N+T][heads][d] bf16 and lse [hq][N+T] are full-size device buffers with
+ * the layouts above; rows a rank does not own are neither read nor written.  `ws`
+ * holds spava_shard_layout.workspace_bytes.  Together the four stages over all
+ * ranks compute spava_attn_prefill_two_stage's result with the score kernel's
+ * scores (spava_attn_prefill's selection). */
+typedef enum {
+  SPAVA_SHARD_SELECT = 0,
+  SPAVA_SHARD_LOCAL = 1,
+  SPAVA_SHARD_REMOTE = 2,
+  SPAVA_SHARD_MERGE = 3
+} spava_shard_stage_id;
+
+spava_status spava_shard_stage(const spava_plan* plan, int32_t stage, const void* q, const void* k,
+                               const void* v, void* o, float* lse, void* ws, void* stream);
+
 /* Synchronise `stream`, read the workspace error word, clear it.  Returns SPAVA_OK,
  * SPAVA_ERR_TIMEOUT (a bounded device wait ran out) or SPAVA_ERR_CUDA. */
 spava_status spava_check_device_error(const spava_plan* plan, void* ws, void* stream);
@@ -293,7 +384,7 @@ spava_status spava_profile_end(spava_plan* plan);
 /* Name of a kernel label: 0 score, 1 select, 2 gather, 3 attention (prefill),
  * 4 lse merge, 5 attention (dense causal), 6 select + gather (fused, prefill),
  * 7 score-key fill/convert (two-stage), 8 attention stage 1, 9 attention stage 2,
- * 10 probe-row lse (probability scores). */
+ * 10 probe-row lse (probability scores), 11 passing unpack (sharded prefill). */
 const char* spava_kernel_name(int32_t label);
 
 /* Static text of a status code. */

@@ -11,6 +11,7 @@ from .spava_oracle import (  # noqa: F401
     approx_attention,
     attention_rows,
     bf16_bits_to_f64,
+    contiguous_owners,
     dense_causal,
     host_of_row,
     host_offsets,
@@ -19,4 +20,6 @@ from .spava_oracle import (  # noqa: F401
     prefill,
     probe_scores,
     select_passing,
+    sharded_attention,
+    zigzag_owners,
 )

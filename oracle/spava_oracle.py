@@ -49,6 +49,9 @@ Readings taken where they are silent (each is a parameter of this oracle):
   R7  ties in selection: larger score first; equal scores -> lower token index;
       -0.0 equals +0.0.  The P chosen indices are stored in ascending order.
   R8  GQA: query head c uses KV head c // (hq / hkv) (parity unpinned).
+  R9  ZigZag arrangement with more than 2W virtual hosts on W ranks: the pairing of
+      rank r with virtual hosts r and 2W-1-r repeats over consecutive rounds of 2W
+      hosts (the pages only describe one round).
 """
 
 from typing import Dict, Optional, Sequence
@@ -316,3 +319,80 @@ def prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, host_sizes: Sequence[in
     else:
         out["O"], out["lse"] = attention_rows(q, k, v, off, anchor, out["sel"], scale, *rows)
     return out
+
+
+def zigzag_owners(n_hosts: int, world: int) -> np.ndarray:
+    """ZigZag arrangement (APB-V technical summary, 1. Framework design, "Context
+    splitting & ZigZag arrangement": a physical host runs the pair of virtual hosts h
+    and 2H-1-h; the German explainer, "Lastverteilung": the first worker takes the
+    first and the last block, the second the second and the one before last, and so
+    on).  Rank of each of n_hosts virtual hosts on ``world`` ranks; reading R9 for
+    n_hosts > 2 * world."""
+    if world < 1 or n_hosts % (2 * world):
+        raise ValueError("zigzag needs n_hosts to be a multiple of 2 * world")
+    owner = np.empty(n_hosts, dtype=np.int64)
+    for h in range(n_hosts):
+        t = h % (2 * world)          # position inside its round of 2W hosts
+        owner[h] = t if t < world else 2 * world - 1 - t
+    return owner
+
+
+def contiguous_owners(n_hosts: int, world: int) -> np.ndarray:
+    """Plain split: rank r runs the n_hosts / world consecutive hosts starting at
+    r * n_hosts / world."""
+    if world < 1 or n_hosts % world:
+        raise ValueError("contiguous split needs n_hosts to be a multiple of world")
+    per = n_hosts // world
+    return np.array([h // per for h in range(n_hosts)], dtype=np.int64)
+
+
+def sharded_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, off: np.ndarray, anchor: int,
+                      sel: np.ndarray, scale: float, owner: Sequence[int]):
+    """The multi-host form of ``approx_attention`` (2. System optimisations, "Fused
+    context and query forward" and the two-stage attention of "Main contributions"):
+    every rank computes, for its own hosts, the rows' attention over the own block
+    (causal) and, separately, over [anchor | passing of earlier hosts], and merges the
+    two through the lse; the text rows get one partial per host block (from the
+    rank owning that host) plus their own causal part (from the owner of the last
+    host), merged through the lse.  Returns (O, lse) like approx_attention; equal to it
+    up to rounding, which pins the decomposition."""
+    NT, hq, d = q.shape
+    hkv = k.shape[1]
+    H = len(off) - 1
+    N = int(off[H])
+    O = np.zeros((NT, hq, d))
+    lse = np.zeros((hq, NT))
+    for c in range(hq):
+        g = sel_row(sel, c, hq, hkv)
+        kv = c // _groups(hq, hkv)
+        for h in range(H):
+            a, e = int(off[h]), int(off[h + 1])
+            rows = np.arange(a, e)
+            logits = np.matmul(q[a:e, c, :], k[a:e, kv, :].T) * scale
+            o_loc, l_loc = _masked_softmax_attend(logits, rows[None, :] <= rows[:, None], v[a:e, kv, :])
+            remote = []
+            if h >= 1:
+                remote = list(range(anchor)) + [int(x) for hh in range(h) for x in sel[hh, g]]
+            if remote:
+                ridx = np.array(remote)
+                logits = np.matmul(q[a:e, c, :], k[ridx, kv, :].T) * scale
+                o_rem, l_rem = _masked_softmax_attend(logits, np.ones(logits.shape, bool), v[ridx, kv, :])
+                o_loc, l_loc = lse_merge(o_loc, l_loc, o_rem, l_rem)
+            O[a:e, c], lse[c, a:e] = o_loc, l_loc
+        if NT > N:
+            rows = np.arange(N, NT)
+            parts = []
+            for h in range(H):
+                a, e = int(off[h]), int(off[h + 1])
+                logits = np.matmul(q[N:NT, c, :], k[a:e, kv, :].T) * scale
+                parts.append((owner[h], _masked_softmax_attend(logits, np.ones(logits.shape, bool), v[a:e, kv, :])))
+            logits = np.matmul(q[N:NT, c, :], k[N:NT, kv, :].T) * scale
+            parts.append((owner[H - 1], _masked_softmax_attend(logits, rows[None, :] <= rows[:, None],
+                                                               v[N:NT, kv, :])))
+            # all ranks' pieces meet after the exchange: merged in rank order
+            parts.sort(key=lambda x: x[0])
+            o_t, l_t = parts[0][1]
+            for _, (op, lp) in parts[1:]:
+                o_t, l_t = lse_merge(o_t, l_t, op, lp)
+            O[N:NT, c], lse[c, N:NT] = o_t, l_t
+    return O, lse

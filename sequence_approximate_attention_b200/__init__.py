@@ -19,7 +19,7 @@ from . import _lib
 from ._lib import SpavaError, load  # noqa: F401
 
 __all__ = ["Plan", "score_select", "gather_passing", "attn_prefill", "attn_prefill_two_stage", "dense_causal",
-           "check_device_error", "SpavaError", "load", "last_launch_count"]
+           "check_device_error", "SpavaError", "load", "last_launch_count", "shard_owners", "shard_stage"]
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -111,6 +111,26 @@ class Plan:
         self.score_kind = kind
         self.workspace_bytes = int(self.lib.spava_workspace_bytes(self._h))
         self.two_stage_workspace_bytes = int(self.lib.spava_two_stage_workspace_bytes(self._h))
+
+    def set_shard(self, rank: int, world: int, owner: Sequence[int]) -> None:
+        """spava_plan_set_shard: this plan runs rank ``rank`` of ``world``, host h on rank
+        owner[h] (the same list on every rank).  Query shard_layout() afterwards."""
+        if len(owner) != self.n_hosts:
+            raise ValueError(f"owner needs one rank per host ({self.n_hosts})")
+        arr = (ctypes.c_int32 * self.n_hosts)(*[int(x) for x in owner])
+        with torch.cuda.device(self.device):
+            _lib.check(self.lib.spava_plan_set_shard(self._h, int(rank), int(world), arr), "spava_plan_set_shard")
+        self.shard_rank, self.shard_world, self.owner = int(rank), int(world), [int(x) for x in owner]
+
+    def shard_layout(self) -> "_lib.ShardLayout":
+        """spava_shard_query: byte offsets of the exchange buffers in the sharded workspace."""
+        out = _lib.ShardLayout()
+        _lib.check(self.lib.spava_shard_query(self._h, ctypes.byref(out)), "spava_shard_query")
+        return out
+
+    def shard_stage(self, stage: int, q, k, v, o, lse, workspace: torch.Tensor, stream=None) -> None:
+        """spava_shard_stage (module function shard_stage) on this plan."""
+        shard_stage(self, stage, q, k, v, o, lse, workspace, stream)
 
     def set_debug(self, wait_limit_ns: int = 0, stall_producer: bool = False) -> None:
         _lib.check(self.lib.spava_plan_set_debug(self._h, int(wait_limit_ns), int(bool(stall_producer))),
@@ -292,6 +312,41 @@ def dense_causal(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                      _ptr(ws), _stream(stream))
     _lib.check(st, "spava_dense_causal")
     return o, lse
+
+
+SHARD_POLICY = {"contiguous": _lib.SPAVA_SHARD_CONTIGUOUS, "zigzag": _lib.SPAVA_SHARD_ZIGZAG}
+
+
+def shard_owners(n_hosts: int, world: int, policy: str = "zigzag"):
+    """spava_shard_owners (host-side, no device): the rank of every host under the
+    "contiguous" or "zigzag" policy."""
+    if policy not in SHARD_POLICY:
+        raise ValueError(f"policy must be one of {sorted(SHARD_POLICY)}")
+    lib = _lib.load()
+    arr = (ctypes.c_int32 * max(int(n_hosts), 1))()
+    _lib.check(lib.spava_shard_owners(int(n_hosts), int(world), SHARD_POLICY[policy], arr), "spava_shard_owners")
+    return [int(arr[h]) for h in range(int(n_hosts))]
+
+
+def shard_stage(plan: Plan, stage: int, q: Optional[torch.Tensor], k: Optional[torch.Tensor],
+                v: Optional[torch.Tensor], o: Optional[torch.Tensor], lse: Optional[torch.Tensor],
+                workspace: torch.Tensor, stream=None) -> None:
+    """spava_shard_stage: one stage (SPAVA_SHARD_SELECT / LOCAL / REMOTE / MERGE) of the
+    sharded prefill on full-size q/k/v/o/lse buffers; see include/spava.h for which rows
+    each stage reads and writes."""
+    dev = plan.device
+    if stage != _lib.SPAVA_SHARD_MERGE:
+        plan._check_qkv(q, k, v)
+    if stage != _lib.SPAVA_SHARD_SELECT:
+        _expect(o, "o", torch.bfloat16, (plan.n_total, plan.hq, plan.head_dim), dev)
+        _expect(lse, "lse", torch.float32, (plan.hq, plan.n_total), dev)
+    need = int(plan.shard_layout().workspace_bytes)
+    if workspace.dtype != torch.uint8 or workspace.numel() < need or workspace.device != dev or \
+            workspace.data_ptr() % 256:
+        raise ValueError(f"workspace: uint8, 256-byte aligned, >= {need} bytes on the plan's device")
+    st = plan.lib.spava_shard_stage(plan.handle, int(stage), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                    _ptr(workspace), _stream(stream))
+    _lib.check(st, "spava_shard_stage")
 
 
 def check_device_error(plan: Plan, workspace: torch.Tensor, stream=None) -> None:

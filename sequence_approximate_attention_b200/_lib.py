@@ -16,6 +16,23 @@ SPAVA_ERR_CUDA = 3
 SPAVA_ERR_TIMEOUT = 4
 SPAVA_SCORES_GIVEN = 1
 
+SPAVA_SHARD_CONTIGUOUS = 0
+SPAVA_SHARD_ZIGZAG = 1
+SPAVA_SHARD_SELECT, SPAVA_SHARD_LOCAL, SPAVA_SHARD_REMOTE, SPAVA_SHARD_MERGE = 0, 1, 2, 3
+
+
+class ShardLayout(ctypes.Structure):
+    """spava_shard_layout (include/spava.h): byte offsets of the sharded prefill's
+    exchange buffers in its workspace."""
+    _fields_ = [("workspace_bytes", ctypes.c_uint64),
+                ("pass_k_offset", ctypes.c_uint64), ("pass_v_offset", ctypes.c_uint64),
+                ("pass_bytes_per_rank", ctypes.c_uint64),
+                ("text_o_offset", ctypes.c_uint64), ("text_o_bytes_per_rank", ctypes.c_uint64),
+                ("text_lse_offset", ctypes.c_uint64), ("text_lse_bytes_per_rank", ctypes.c_uint64),
+                ("scores_offset", ctypes.c_uint64), ("idx_offset", ctypes.c_uint64),
+                ("pass_slots", c_int32), ("text_slots", c_int32)]
+
+
 # name -> (restype, argtypes); the names and order follow include/spava.h.
 SIGNATURES = {
     "spava_plan_create": (c_int32, [ctypes.POINTER(c_void_p), c_int32, c_int32, c_int32,
@@ -37,6 +54,11 @@ SIGNATURES = {
     "spava_two_stage_workspace_bytes": (c_size_t, [c_void_p]),
     "spava_dense_causal": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                      c_void_p, c_void_p, c_void_p]),
+    "spava_shard_owners": (c_int32, [c_int32, c_int32, c_int32, ctypes.POINTER(c_int32)]),
+    "spava_plan_set_shard": (c_int32, [c_void_p, c_int32, c_int32, ctypes.POINTER(c_int32)]),
+    "spava_shard_query": (c_int32, [c_void_p, ctypes.POINTER(ShardLayout)]),
+    "spava_shard_stage": (c_int32, [c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                    c_void_p, c_void_p]),
     "spava_check_device_error": (c_int32, [c_void_p, c_void_p, c_void_p]),
     "spava_plan_set_debug": (c_int32, [c_void_p, ctypes.c_uint64, c_int32]),
     "spava_plan_set_score_reduce": (c_int32, [c_void_p, c_int32]),

@@ -38,7 +38,8 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
 }
 
 // One CTA per (host h < H-1, selection row g: a KV head, or a query head with
-// per-query-head selection).  Candidates: [off[h] + (h == 0 ? A : 0),
+// per-query-head selection); with a host list, CTA (s, g) takes host hosts[s]
+// (the sharded prefill: a rank's own hosts), else host s.  Candidates: [off[h] + (h == 0 ? A : 0),
 // off[h+1]).  Radix select (four 8-bit digits, most significant first) finds the
 // P-th largest key T and how many keys equal to T are taken; a stable compaction in
 // index order then writes the P winners ascending: keys > T, and the lowest-index
@@ -46,8 +47,8 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
 // Thread t owns the contiguous keys [t*per, (t+1)*per).  With kPer > 0 they are read
 // once into registers (segments up to kPer * blockDim.x keys); kPer == 0 re-reads
 // them from global memory on every pass (any segment length).
-// With kGather the CTA then copies its P passing rows of K and V into
-// k_pass/v_pass[g][h] (16 bytes per thread), so the prefill needs no separate gather.
+// With kGather the CTA then copies its P passing rows of K and V into host slot s
+// of the destination (16 bytes per thread), so the prefill needs no separate gather.
 constexpr int kGatherUnroll = 4;
 
 struct GatherArgs {
@@ -55,20 +56,27 @@ struct GatherArgs {
   const uint4* v;
   uint4* kp;
   uint4* vp;
-  int hosts_m1;
   int chunks_per_row;  // 16-byte chunks per K/V row (d * 2 / 16)
   int kv_heads;        // hkv (row stride of k and v)
   int group_div;       // selection row r reads KV head r / group_div (1, or G per query head)
+  // Destination of passing row j of selection row g in host slot s, in 16-byte
+  // chunks: kp + g * dst_g + s * dst_h + j * dst_j.  k_pass/v_pass[g][h][j] has
+  // dst_j = chunks_per_row, dst_h = P * dst_j, dst_g = (H-1) * dst_h; the rank-major
+  // exchange buffer of the sharded prefill, [slot][j][g], has dst_g = chunks_per_row,
+  // dst_j = rows * chunks_per_row, dst_h = P * dst_j.
+  size_t dst_g, dst_h, dst_j;
 };
 
 template <int kPer, bool kGather>
 __global__ void __launch_bounds__(1024) select_topp_kernel(const float* __restrict__ scores, int n_visual,
                                                             const int* __restrict__ off, int anchor, int passing,
-                                                            int rows, int32_t* __restrict__ idx, GatherArgs ga) {
+                                                            int rows, const int* __restrict__ hosts,
+                                                            int32_t* __restrict__ idx, GatherArgs ga) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t scan_scratch[33];
   __shared__ uint32_t sh_prefix, sh_k;
-  const int h = blockIdx.x / rows, g = blockIdx.x % rows;
+  const int slot = blockIdx.x / rows, g = blockIdx.x % rows;
+  const int h = hosts ? hosts[slot] : slot;
   const int lo = off[h] + (h == 0 ? anchor : 0), hi = off[h + 1];
   const int n = hi - lo;
   const float* s = scores + static_cast<size_t>(g) * n_visual + lo;
@@ -168,7 +176,7 @@ __global__ void __launch_bounds__(1024) select_topp_kernel(const float* __restri
     const int cpr = ga.chunks_per_row;  // a power of two (8 or 16)
     const int cpr_shift = __ffs(cpr) - 1;
     const int total = passing * cpr;
-    const size_t dst0 = ((static_cast<size_t>(g) * ga.hosts_m1 + h) * passing) * cpr;
+    const size_t dst0 = static_cast<size_t>(g) * ga.dst_g + static_cast<size_t>(slot) * ga.dst_h;
     const int kvh = g / ga.group_div;
     for (int t0 = tid; t0 < total; t0 += kGatherUnroll * nt) {
       uint4 kv[kGatherUnroll], vv[kGatherUnroll];
@@ -186,8 +194,9 @@ __global__ void __launch_bounds__(1024) select_topp_kernel(const float* __restri
       for (int u = 0; u < kGatherUnroll; ++u) {
         const int t = t0 + u * nt;
         if (t < total) {
-          ga.kp[dst0 + t] = kv[u];
-          ga.vp[dst0 + t] = vv[u];
+          const size_t dst = dst0 + static_cast<size_t>(t >> cpr_shift) * ga.dst_j + (t & (cpr - 1));
+          ga.kp[dst] = kv[u];
+          ga.vp[dst] = vv[u];
         }
       }
     }
@@ -244,6 +253,30 @@ __global__ void __launch_bounds__(256) gather_passing_kernel(const uint4* __rest
     const size_t src = (static_cast<size_t>(tok) * kv_heads + g / group_div) * chunks_per_row + ch;
     kp[t] = __ldg(k + src);
     vp[t] = __ldg(v + src);
+  }
+}
+
+// Sharded prefill: the passing rows of every host, from the rank-major exchange
+// buffer that the ranks' selections filled (row j of host h's slot, selection row g,
+// at x[(xrow0[h] + j) * rows + g]), into k_pass/v_pass[g][h][j][:].
+__global__ void __launch_bounds__(256) unpack_passing_kernel(const uint4* __restrict__ xk,
+                                                              const uint4* __restrict__ xv,
+                                                              const int* __restrict__ xrow0, uint4* __restrict__ kp,
+                                                              uint4* __restrict__ vp, int rows, int hosts_m1,
+                                                              int passing, int chunks_per_row) {
+  const size_t rows_per_g = static_cast<size_t>(hosts_m1) * passing;
+  const size_t total = static_cast<size_t>(rows) * rows_per_g * chunks_per_row;
+  for (size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t r = t / chunks_per_row;
+    const int ch = static_cast<int>(t - r * chunks_per_row);
+    const int g = static_cast<int>(r / rows_per_g);
+    const size_t rem = r - static_cast<size_t>(g) * rows_per_g;
+    const int h = static_cast<int>(rem / passing);
+    const int j = static_cast<int>(rem - static_cast<size_t>(h) * passing);
+    const size_t src = ((static_cast<size_t>(__ldg(xrow0 + h)) + j) * rows + g) * chunks_per_row + ch;
+    kp[t] = __ldg(xk + src);
+    vp[t] = __ldg(xv + src);
   }
 }
 

@@ -120,10 +120,29 @@ struct spava_plan {
   int n_score_pre = 0;
   int4* d_score_all = nullptr;  // all hosts
   int n_score_all = 0;
+  // sharded prefill (spava_plan_set_shard): this rank's work lists in their own
+  // device table; the exchange buffers' slots per rank
+  int shard_rank = 0, shard_world = 0;  // world 0: not sharded
+  std::vector<int> owner;               // rank of each host
+  int pass_slots = 0, text_slots = 0;   // per rank
+  int text_slots_used = 0;              // this rank's text pieces
+  void* dtab_shard = nullptr;
+  int* d_shard_hosts = nullptr;  // own hosts < H-1, ascending: the select grid's host list
+  int n_shard_hosts = 0;
+  int* d_xrow0 = nullptr;        // [H-1] first exchange row of each host's passing rows
+  int4* d_score_shard = nullptr;
+  int n_score_shard = 0;
+  AttnItem* d_items_shard_local = nullptr;
+  int n_items_shard_local = 0;
+  AttnItem* d_items_shard_remote = nullptr;
+  int n_items_shard_remote = 0;
+  AttnItem* d_items_shard_probe = nullptr;
+  int n_items_shard_probe = 0;
   // workspace layout
   size_t ws_err = 0, ws_scores = 0, ws_idx = 0, ws_kp = 0, ws_vp = 0, ws_opart = 0, ws_lpart = 0, ws_total = 0;
   size_t ws_row_o = 0, ws_row_lse = 0, ws_qkeys = 0, ws_total_two_stage = 0;  // two-stage flow only
   size_t ws_probe_lse = 0;  // probability scores: [hq][N] lse (probe rows only)
+  size_t ws_xk = 0, ws_xv = 0, ws_to = 0, ws_tl = 0, ws_total_shard = 0;  // sharded prefill
   // debug knobs
   uint64_t wait_limit_ns = spava::kDefaultWaitLimitNs;
   int stall_producer = 0;
@@ -140,7 +159,7 @@ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 enum KernelLabel {
   kLabScore = 0, kLabSelect = 1, kLabGather = 2, kLabAttn = 3, kLabMerge = 4, kLabDense = 5, kLabSelectGather = 6,
-  kLabFill = 7, kLabAttnLocal = 8, kLabAttnRemote = 9, kLabProbeLse = 10
+  kLabFill = 7, kLabAttnLocal = 8, kLabAttnRemote = 9, kLabProbeLse = 10, kLabUnpack = 11
 };
 
 void mark(const spava_plan* p, int label, cudaStream_t st) {
@@ -193,14 +212,24 @@ AttnItem blank_item(int q_row0, int q_rows, int q_head, int out) {
   return it;
 }
 
-// Text-query pieces of the prefill (shared by both flows): T rows in 256-row items,
-// split over the host blocks plus their own causal part, each an fp32 partial.
-void add_text_items(const spava_plan& p, std::vector<AttnItem>& v, std::vector<int>& group) {
+// Which hosts a work list covers: every host (nullptr), or one rank's hosts in the
+// sharded prefill.
+using HostMask = std::vector<char>;
+bool runs(const HostMask* mine, int h) { return !mine || (*mine)[h] != 0; }
+
+// Text-query pieces of the prefill (shared by all flows): T rows in 256-row items,
+// split over the host blocks (piece k < H) plus their own causal part (piece H),
+// each an fp32 partial into slot k, or into slot[k] when a slot map is given
+// (pieces with slot -1 belong to other ranks).
+void add_text_items(const spava_plan& p, std::vector<AttnItem>& v, std::vector<int>& group,
+                    const std::vector<int>* slot = nullptr) {
   for (int r0 = p.N; r0 < p.N + p.T; r0 += 256) {
     const int rows = std::min(256, p.N + p.T - r0);
     for (int c = 0; c < p.hq; ++c) {
       for (int k = 0; k <= p.H; ++k) {
-        AttnItem it = blank_item(r0, rows, c, spava::make_out(spava::kOutTextPartial, k));
+        const int sl = slot ? (*slot)[k] : k;
+        if (sl < 0) continue;
+        AttnItem it = blank_item(r0, rows, c, spava::make_out(spava::kOutTextPartial, sl));
         if (k < p.H)
           it.seg[0] = AttnSeg{p.off[k], p.off[k + 1] - p.off[k], 0, 0};
         else
@@ -244,16 +273,18 @@ bool scores_needed(const spava_plan& p) { return p.H >= 2 && p.P > 0; }
 
 // Two-stage flow, first launch: every host's queries over its own block (causal).
 // Hosts with a remote part write fp32 partials of their rows; items holding probe
-// rows of hosts < H-1 also fold their logits into the probe scores.  Text pieces
-// run here too.
-std::vector<AttnItem> build_local_items(const spava_plan& p) {
+// rows of hosts < H-1 also fold their logits into the probe scores (one GPU; the
+// sharded prefill scores with the score kernel first).  Text pieces run here too.
+std::vector<AttnItem> build_local_items(const spava_plan& p, const HostMask* mine = nullptr,
+                                        const std::vector<int>* text_slot = nullptr) {
   std::vector<AttnItem> v;
   std::vector<int> group;
   for (int h = 0; h < p.H; ++h) {
+    if (!runs(mine, h)) continue;
     const int a = p.off[h], e = p.off[h + 1];
     for (int r0 = a; r0 < e; r0 += 256) {
       const int rows = std::min(256, e - r0);
-      const bool probe = scores_needed(p) && h < p.H - 1 && r0 + rows > e - p.R;
+      const bool probe = !mine && scores_needed(p) && h < p.H - 1 && r0 + rows > e - p.R;
       const int mode = has_remote(p, h) ? spava::kOutRowPartial : spava::kOutFinal;
       for (int c = 0; c < p.hq; ++c) {
         AttnItem it = blank_item(r0, rows, c, spava::make_out(mode, 0, probe));
@@ -263,18 +294,18 @@ std::vector<AttnItem> build_local_items(const spava_plan& p) {
       }
     }
   }
-  add_text_items(p, v, group);
+  add_text_items(p, v, group, text_slot);
   sort_host_major(v, group, p.hq / p.hkv);
   return v;
 }
 
 // Two-stage flow, second launch: host h >= 1 over [anchor | passing of hosts < h],
 // lse-merged with its local partial into the final output.
-std::vector<AttnItem> build_remote_items(const spava_plan& p) {
+std::vector<AttnItem> build_remote_items(const spava_plan& p, const HostMask* mine = nullptr) {
   std::vector<AttnItem> v;
   std::vector<int> group;
   for (int h = 1; h < p.H; ++h) {
-    if (!has_remote(p, h)) continue;
+    if (!has_remote(p, h) || !runs(mine, h)) continue;
     const int a = p.off[h], e = p.off[h + 1];
     for (int r0 = a; r0 < e; r0 += 256) {
       const int rows = std::min(256, e - r0);
@@ -292,13 +323,14 @@ std::vector<AttnItem> build_remote_items(const spava_plan& p) {
   return v;
 }
 
-// Probability scores: the last R rows of every host over its own block (causal), lse
-// only -- each probe row's log-sum-exp over the keys of its block it sees.
-std::vector<AttnItem> build_probe_items(const spava_plan& p) {
+// Probability scores: the last R rows of every host h < h_end over its own block
+// (causal), lse only -- each probe row's log-sum-exp over the keys of its block it sees.
+std::vector<AttnItem> build_probe_items(const spava_plan& p, int h_end, const HostMask* mine = nullptr) {
   std::vector<AttnItem> v;
   std::vector<int> group;
   if (p.R == 0) return v;
-  for (int h = 0; h < p.H; ++h) {
+  for (int h = 0; h < h_end; ++h) {
+    if (!runs(mine, h)) continue;
     const int a = p.off[h], e = p.off[h + 1];
     for (int r0 = e - p.R; r0 < e; r0 += 256) {
       const int rows = std::min(256, e - r0);
@@ -329,11 +361,12 @@ std::vector<AttnItem> build_dense_items(const spava_plan& p) {
   return v;
 }
 
-std::vector<int4> build_score_items(const spava_plan& p, int h_end) {
+std::vector<int4> build_score_items(const spava_plan& p, int h_end, const HostMask* mine = nullptr) {
   std::vector<int4> v;
   for (int h = 0; h < h_end; ++h)
-    for (int g = 0; g < p.hkv; ++g)
-      for (int k0 = p.off[h]; k0 < p.off[h + 1]; k0 += 128) v.push_back(make_int4(h, g, k0, p.off[h + 1]));
+    if (runs(mine, h))
+      for (int g = 0; g < p.hkv; ++g)
+        for (int k0 = p.off[h]; k0 < p.off[h + 1]; k0 += 128) v.push_back(make_int4(h, g, k0, p.off[h + 1]));
   return v;
 }
 
@@ -382,6 +415,17 @@ void layout_workspace(spava_plan* p) {
   p->ws_qkeys = o;  // per-query-head score keys (all but the max head reduction)
   o = align_up(o + hq * n_visual * 4, 256);
   p->ws_total_two_stage = o;
+  // Sharded prefill: rank-major exchange buffers, each rank's part one contiguous run.
+  const size_t world = static_cast<size_t>(p->shard_world);
+  p->ws_xk = o;
+  o = align_up(o + world * p->pass_slots * P * rows * d * 2, 256);
+  p->ws_xv = o;
+  o = align_up(o + world * p->pass_slots * P * rows * d * 2, 256);
+  p->ws_to = o;
+  o = align_up(o + world * p->text_slots * n_text * hq * d * 4, 256);
+  p->ws_tl = o;
+  o = align_up(o + world * p->text_slots * hq * n_text * 4, 256);
+  p->ws_total_shard = o;
 }
 
 spava_status check_plan_ws(const spava_plan* p, void* ws) {
@@ -393,9 +437,8 @@ spava_status check_plan_ws(const spava_plan* p, void* ws) {
 
 // ------------------------------------------------------------------ launches
 template <int D>
-spava_status launch_score(const spava_plan* p, const void* q, const void* k, float* scores, bool all_hosts,
-                          void* ws, cudaStream_t st) {
-  const int n_items = all_hosts ? p->n_score_all : p->n_score_pre;
+spava_status launch_score(const spava_plan* p, const void* q, const void* k, float* scores, const int4* items,
+                          int n_items, void* ws, cudaStream_t st) {
   if (n_items == 0) return SPAVA_OK;
   CUtensorMap tmK, tmQp;
   spava_status s;
@@ -403,7 +446,7 @@ spava_status launch_score(const spava_plan* p, const void* q, const void* k, flo
   const int G = p->hq / p->hkv;
   if ((s = make_map(&tmQp, q, D, p->hq, p->N + p->T, 1, p->rc)) != SPAVA_OK) return s;
   ScoreParams sp;
-  sp.items = all_hosts ? p->d_score_all : p->d_score_pre;
+  sp.items = items;
   sp.n_items = n_items;
   sp.probe_r = p->R;
   sp.group = G;
@@ -439,29 +482,55 @@ spava_status launch_score(const spava_plan* p, const void* q, const void* k, flo
   return SPAVA_OK;
 }
 
-// Top-P selection; with k/v/kp/vp given, each selection CTA also gathers its passing
-// rows (the prefill's fused select + gather).
+// Where a fused selection writes its passing rows: k_pass/v_pass[g][h][j] (one GPU),
+// or this rank's part of the rank-major exchange buffers [slot][j][g] (sharded).
+struct PassDest {
+  void* kp = nullptr;
+  void* vp = nullptr;
+  bool exchange = false;
+};
+
+// Top-P selection of hosts 0..H-2, or of the hosts in `hosts` (device list of
+// n_hosts); with k/v and a destination given, each selection CTA also gathers its
+// passing rows (the prefill's fused select + gather).
 spava_status launch_select(const spava_plan* p, const float* scores, int32_t* idx, cudaStream_t st,
-                           const void* k = nullptr, const void* v = nullptr, void* kp = nullptr, void* vp = nullptr) {
+                           const void* k = nullptr, const void* v = nullptr, PassDest dst = PassDest(),
+                           const int* hosts = nullptr, int n_hosts = -1) {
   if (p->H < 2 || p->P == 0) return SPAVA_OK;
+  if (n_hosts < 0) n_hosts = p->H - 1;
+  if (n_hosts == 0) return SPAVA_OK;
   int max_seg = 0;
   for (int h = 0; h + 1 < p->H; ++h) max_seg = std::max(max_seg, p->off[h + 1] - p->off[h]);
   const int rows = score_rows(*p);
-  spava::GatherArgs ga{static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(kp),
-                       static_cast<uint4*>(vp), p->H - 1, p->d * 2 / 16, p->hkv, rows / p->hkv};
+  const size_t cpr = static_cast<size_t>(p->d) * 2 / 16;
+  spava::GatherArgs ga{static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(dst.kp),
+                       static_cast<uint4*>(dst.vp), static_cast<int>(cpr), p->hkv, rows / p->hkv, 0, 0, 0};
+  if (dst.exchange) {
+    ga.dst_g = cpr;
+    ga.dst_j = rows * cpr;
+    ga.dst_h = static_cast<size_t>(p->P) * ga.dst_j;
+  } else {
+    ga.dst_j = cpr;
+    ga.dst_h = static_cast<size_t>(p->P) * cpr;
+    ga.dst_g = static_cast<size_t>(p->H - 1) * ga.dst_h;
+  }
   const bool fused = k != nullptr;
-  const int grid = (p->H - 1) * rows;
+  const int grid = n_hosts * rows;
   mark(p, fused ? kLabSelectGather : kLabSelect, st);
   if (max_seg <= 16 * 1024) {
     if (fused)
-      spava::select_topp_kernel<16, true><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, rows, idx, ga);
+      spava::select_topp_kernel<16, true><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, rows, hosts,
+                                                                  idx, ga);
     else
-      spava::select_topp_kernel<16, false><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, rows, idx, ga);
+      spava::select_topp_kernel<16, false><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, rows, hosts,
+                                                                   idx, ga);
   } else {
     if (fused)
-      spava::select_topp_kernel<0, true><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, rows, idx, ga);
+      spava::select_topp_kernel<0, true><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, rows, hosts,
+                                                                 idx, ga);
     else
-      spava::select_topp_kernel<0, false><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, rows, idx, ga);
+      spava::select_topp_kernel<0, false><<<grid, 1024, 0, st>>>(scores, p->N, p->d_off, p->A, p->P, rows, hosts,
+                                                                  idx, ga);
   }
   SPAVA_CUDA(cudaGetLastError());
   ++g_last_launches;
@@ -490,6 +559,8 @@ struct TwoStageBufs {
   float* row_lse = nullptr;
   unsigned int* score_keys = nullptr;
   int per_qhead = 0;  // score_keys has one row per query head
+  float* text_o = nullptr;    // text partial slots elsewhere than the workspace's
+  float* text_lse = nullptr;  // (the sharded prefill's exchange buffers)
 };
 
 template <int D>
@@ -521,8 +592,8 @@ spava_status launch_attn(const spava_plan* p, const AttnItem* items, int n_items
   ap.o = static_cast<__nv_bfloat16*>(o);
   ap.lse = lse;
   uint8_t* w = static_cast<uint8_t*>(ws);
-  ap.o_part = reinterpret_cast<float*>(w + p->ws_opart);
-  ap.lse_part = reinterpret_cast<float*>(w + p->ws_lpart);
+  ap.o_part = ts.text_o ? ts.text_o : reinterpret_cast<float*>(w + p->ws_opart);
+  ap.lse_part = ts.text_lse ? ts.text_lse : reinterpret_cast<float*>(w + p->ws_lpart);
   ap.part_row0 = p->N;
   ap.part_rows = p->T;
   ap.scale_log2 = p->scale * 1.4426950408889634f;
@@ -540,9 +611,9 @@ spava_status launch_attn(const spava_plan* p, const AttnItem* items, int n_items
   if ((s = ensure_smem(spava::attn_fwd_kernel<D>, S::kSmemBytes)) != SPAVA_OK) return s;
   const int grid = std::min(n_items, p->num_sms);
   mark(p, items == p->d_items_dense ? kLabDense
-             : items == p->d_items_local ? kLabAttnLocal
-             : items == p->d_items_remote ? kLabAttnRemote
-             : items == p->d_items_probe ? kLabProbeLse : kLabAttn, st);
+             : (items == p->d_items_local || items == p->d_items_shard_local) ? kLabAttnLocal
+             : (items == p->d_items_remote || items == p->d_items_shard_remote) ? kLabAttnRemote
+             : (items == p->d_items_probe || items == p->d_items_shard_probe) ? kLabProbeLse : kLabAttn, st);
   spava::attn_fwd_kernel<D><<<grid, S::kThreads, S::kSmemBytes, st>>>(tmQ, tmK, tmV, tmKp, tmVp, ap);
   SPAVA_CUDA(cudaGetLastError());
   ++g_last_launches;
@@ -552,39 +623,76 @@ spava_status launch_attn(const spava_plan* p, const AttnItem* items, int n_items
 // Probability scores: the lse of every host's probe rows over its block, into the
 // workspace (the items' O is not stored; V only has to be a readable K/V tensor).
 spava_status launch_probe_lse(const spava_plan* p, const void* q, const void* k, const void* v, void* ws,
-                              cudaStream_t st) {
+                              cudaStream_t st, const AttnItem* items = nullptr, int n_items = -1) {
   if (p->score_kind != SPAVA_SCORE_PROB) return SPAVA_OK;
+  if (!items) {
+    items = p->d_items_probe;
+    n_items = p->n_items_probe;
+  }
   TwoStageBufs t;
   t.row_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + p->ws_probe_lse);
-  return p->d == 128 ? launch_attn<128>(p, p->d_items_probe, p->n_items_probe, q, k, v, nullptr, nullptr, nullptr,
-                                        nullptr, ws, st, t)
-                     : launch_attn<64>(p, p->d_items_probe, p->n_items_probe, q, k, v, nullptr, nullptr, nullptr,
-                                       nullptr, ws, st, t);
+  return p->d == 128 ? launch_attn<128>(p, items, n_items, q, k, v, nullptr, nullptr, nullptr, nullptr, ws, st, t)
+                     : launch_attn<64>(p, items, n_items, q, k, v, nullptr, nullptr, nullptr, nullptr, ws, st, t);
 }
 
-spava_status launch_merge(const spava_plan* p, void* o, float* lse, void* ws, cudaStream_t st) {
+// Text rows from n_slots partial slots (the workspace's H+1, or the sharded prefill's
+// gathered world * slots-per-rank).
+spava_status launch_merge(const spava_plan* p, void* o, float* lse, void* ws, cudaStream_t st,
+                          const float* o_part = nullptr, const float* lse_part = nullptr, int n_slots = -1) {
   if (p->T == 0) return SPAVA_OK;
   uint8_t* w = static_cast<uint8_t*>(ws);
+  if (!o_part) {
+    o_part = reinterpret_cast<const float*>(w + p->ws_opart);
+    lse_part = reinterpret_cast<const float*>(w + p->ws_lpart);
+    n_slots = p->H + 1;
+  }
   const int warps = p->T * p->hq;
   const int grid = (warps * 32 + 255) / 256;
   mark(p, kLabMerge, st);
-  spava::lse_merge_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(w + p->ws_opart),
-                                                 reinterpret_cast<const float*>(w + p->ws_lpart), p->H + 1, p->T,
-                                                 p->hq, p->d, p->N, p->N + p->T, static_cast<__nv_bfloat16*>(o), lse);
+  spava::lse_merge_kernel<<<grid, 256, 0, st>>>(o_part, lse_part, n_slots, p->T, p->hq, p->d, p->N, p->N + p->T,
+                                                 static_cast<__nv_bfloat16*>(o), lse);
   SPAVA_CUDA(cudaGetLastError());
   ++g_last_launches;
   return SPAVA_OK;
 }
 
-spava_status begin_call(const spava_plan* p, void* ws, cudaStream_t st) {
+spava_status begin_call(const spava_plan* p, void* ws, cudaStream_t st, bool clear_error = true) {
   g_last_launches = 0;
   ++p->prof_call_id;
   int dev = -1;
   SPAVA_CUDA(cudaGetDevice(&dev));
   if (dev != p->device) return fail(SPAVA_ERR_INVALID_ARG, "current device %d differs from the plan's device %d", dev, p->device);
-  SPAVA_CUDA(cudaMemsetAsync(err_word(p, ws), 0, 256, st));
+  if (clear_error) SPAVA_CUDA(cudaMemsetAsync(err_word(p, ws), 0, 256, st));
   return SPAVA_OK;
 }
+
+// Upload `host` (built with the same put() packing as the plan table) to a fresh
+// device allocation.
+spava_status upload_table(const std::vector<uint8_t>& host, void** out) {
+  *out = nullptr;
+  if (host.empty()) return SPAVA_OK;
+  cudaError_t e = cudaMalloc(out, host.size());
+  if (e != cudaSuccess) return fail(SPAVA_ERR_CUDA, "cudaMalloc(plan table): %s", cudaGetErrorString(e));
+  e = cudaMemcpy(*out, host.data(), host.size(), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(*out);
+    *out = nullptr;
+    return fail(SPAVA_ERR_CUDA, "cudaMemcpy(plan table): %s", cudaGetErrorString(e));
+  }
+  return SPAVA_OK;
+}
+
+// Packs arrays into one host image for upload_table, each 256-byte aligned.
+struct TablePacker {
+  std::vector<uint8_t> host;
+  size_t put(const void* src, size_t bytes) {
+    const size_t at = host.size();
+    const uint8_t* b = static_cast<const uint8_t*>(src);
+    if (bytes) host.insert(host.end(), b, b + bytes);
+    host.resize(align_up(host.size(), 256), 0);
+    return at;
+  }
+};
 
 }  // namespace
 
@@ -681,7 +789,7 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   const auto dense = build_dense_items(*p);
   const auto local = build_local_items(*p);
   const auto remote = build_remote_items(*p);
-  const auto probe = build_probe_items(*p);
+  const auto probe = build_probe_items(*p, n_hosts);
   const auto sc_pre = build_score_items(*p, n_hosts - 1);
   const auto sc_all = build_score_items(*p, n_hosts);
   p->n_items_pre = static_cast<int>(pre.size());
@@ -728,9 +836,10 @@ spava_status spava_plan_destroy(spava_plan* p) {
   if (!p) return ok();
   spava_status s = SPAVA_OK;
   for (cudaEvent_t e : p->prof_ev) cudaEventDestroy(e);
-  if (p->dtab) {
+  if (p->dtab || p->dtab_shard) {
     cudaError_t e = cudaDeviceSynchronize();
-    if (e == cudaSuccess) e = cudaFree(p->dtab);
+    if (e == cudaSuccess && p->dtab) e = cudaFree(p->dtab);
+    if (e == cudaSuccess && p->dtab_shard) e = cudaFree(p->dtab_shard);
     if (e != cudaSuccess) s = fail(SPAVA_ERR_CUDA, "plan destroy: %s", cudaGetErrorString(e));
   }
   delete p;
@@ -786,7 +895,8 @@ spava_status spava_score_select(const spava_plan* p, const void* q, const void* 
   if (!(flags & SPAVA_SCORES_GIVEN) && p->H >= 1) {
     if (p->R == 0) return fail(SPAVA_ERR_INVALID_ARG, "plan has R = 0: nothing to score");
     if ((s = launch_probe_lse(p, q, k, k, ws, st)) != SPAVA_OK) return s;
-    s = p->d == 128 ? launch_score<128>(p, q, k, scores, true, ws, st) : launch_score<64>(p, q, k, scores, true, ws, st);
+    s = p->d == 128 ? launch_score<128>(p, q, k, scores, p->d_score_all, p->n_score_all, ws, st)
+                    : launch_score<64>(p, q, k, scores, p->d_score_all, p->n_score_all, ws, st);
     if (s != SPAVA_OK) return s;
   }
   if ((s = launch_select(p, scores, idx, st)) != SPAVA_OK) return s;
@@ -824,9 +934,10 @@ spava_status spava_attn_prefill(const spava_plan* p, const void* q, const void* 
   void* vp = w + p->ws_vp;
   if (p->H >= 2 && p->P > 0) {
     if ((s = launch_probe_lse(p, q, k, v, ws, st)) != SPAVA_OK) return s;
-    s = p->d == 128 ? launch_score<128>(p, q, k, scores, false, ws, st) : launch_score<64>(p, q, k, scores, false, ws, st);
+    s = p->d == 128 ? launch_score<128>(p, q, k, scores, p->d_score_pre, p->n_score_pre, ws, st)
+                    : launch_score<64>(p, q, k, scores, p->d_score_pre, p->n_score_pre, ws, st);
     if (s != SPAVA_OK) return s;
-    if ((s = launch_select(p, scores, idx, st, k, v, kp, vp)) != SPAVA_OK) return s;
+    if ((s = launch_select(p, scores, idx, st, k, v, PassDest{kp, vp, false})) != SPAVA_OK) return s;
   }
   s = p->d == 128 ? launch_attn<128>(p, p->d_items_pre, p->n_items_pre, q, k, v, kp, vp, o, lse, ws, st)
                   : launch_attn<64>(p, p->d_items_pre, p->n_items_pre, q, k, v, kp, vp, o, lse, ws, st);
@@ -918,7 +1029,8 @@ spava_status spava_attn_prefill_two_stage(const spava_plan* p, const void* q, co
   const int grid_small = std::max(1, std::min(p->num_sms * 4, static_cast<int>((n_keys + 255) / 256)));
   if (scores_needed(*p) && prob) {
     if ((s = launch_probe_lse(p, q, k, v, ws, st)) != SPAVA_OK) return s;
-    s = p->d == 128 ? launch_score<128>(p, q, k, scores, false, ws, st) : launch_score<64>(p, q, k, scores, false, ws, st);
+    s = p->d == 128 ? launch_score<128>(p, q, k, scores, p->d_score_pre, p->n_score_pre, ws, st)
+                    : launch_score<64>(p, q, k, scores, p->d_score_pre, p->n_score_pre, ws, st);
     if (s != SPAVA_OK) return s;
   } else if (scores_needed(*p)) {
     mark(p, kLabFill, st);
@@ -944,7 +1056,7 @@ spava_status spava_attn_prefill_two_stage(const spava_plan* p, const void* q, co
       SPAVA_CUDA(cudaGetLastError());
       ++g_last_launches;
     }
-    if ((s = launch_select(p, scores, idx, st, k, v, kp, vp)) != SPAVA_OK) return s;
+    if ((s = launch_select(p, scores, idx, st, k, v, PassDest{kp, vp, false})) != SPAVA_OK) return s;
   }
   // stage 2: remote pass over [anchor | passing], lse-merged with the local partials
   s = p->d == 128 ? launch_attn<128>(p, p->d_items_remote, p->n_items_remote, q, k, v, kp, vp, o, lse, ws, st, ts)
@@ -967,6 +1079,207 @@ spava_status spava_dense_causal(const spava_plan* p, const void* q, const void* 
   s = p->d == 128 ? launch_attn<128>(p, p->d_items_dense, p->n_items_dense, q, k, v, nullptr, nullptr, o, lse, ws, st)
                   : launch_attn<64>(p, p->d_items_dense, p->n_items_dense, q, k, v, nullptr, nullptr, o, lse, ws, st);
   if (s != SPAVA_OK) return s;
+  mark(p, -1, st);
+  return ok();
+}
+
+spava_status spava_shard_owners(int32_t n_hosts, int32_t world, int32_t policy, int32_t* owner_out) {
+  if (!owner_out || n_hosts < 1 || world < 1) return fail(SPAVA_ERR_INVALID_ARG, "need H >= 1, world >= 1, an array");
+  if (policy == SPAVA_SHARD_CONTIGUOUS) {
+    if (n_hosts % world) return fail(SPAVA_ERR_INVALID_ARG, "contiguous split needs H %% world == 0");
+    const int per = n_hosts / world;
+    for (int h = 0; h < n_hosts; ++h) owner_out[h] = h / per;
+    return ok();
+  }
+  if (policy == SPAVA_SHARD_ZIGZAG) {
+    if (n_hosts % (2 * world)) return fail(SPAVA_ERR_INVALID_ARG, "zigzag needs H %% (2 * world) == 0");
+    for (int h = 0; h < n_hosts; ++h) {
+      const int t = h % (2 * world);
+      owner_out[h] = t < world ? t : 2 * world - 1 - t;
+    }
+    return ok();
+  }
+  return fail(SPAVA_ERR_INVALID_ARG, "unknown shard policy %d", policy);
+}
+
+spava_status spava_plan_set_shard(spava_plan* p, int32_t rank, int32_t world, const int32_t* owner) {
+  if (!p || !owner) return fail(SPAVA_ERR_INVALID_ARG, "plan and owner must not be NULL");
+  if (world < 1 || rank < 0 || rank >= world) return fail(SPAVA_ERR_INVALID_ARG, "need 0 <= rank < world");
+  for (int h = 0; h < p->H; ++h)
+    if (owner[h] < 0 || owner[h] >= world) return fail(SPAVA_ERR_INVALID_ARG, "host %d has owner %d", h, owner[h]);
+  const int H = p->H;
+  const bool passing = scores_needed(*p);
+  // slots: passing rows of each rank's hosts < H-1, text pieces of each rank
+  std::vector<int> n_pass(world, 0), n_text(world, 0), pslot(H, -1);
+  for (int h = 0; h < H; ++h) {
+    if (passing && h < H - 1) pslot[h] = n_pass[owner[h]]++;
+    if (p->T > 0) ++n_text[owner[h]];
+  }
+  if (p->T > 0) ++n_text[owner[H - 1]];  // the text rows' own causal piece
+  const int pass_slots = *std::max_element(n_pass.begin(), n_pass.end());
+  const int text_slots = *std::max_element(n_text.begin(), n_text.end());
+  HostMask mine(H, 0);
+  for (int h = 0; h < H; ++h) mine[h] = owner[h] == rank;
+  std::vector<int> tslot(H + 1, -1);
+  int used = 0;
+  if (p->T > 0) {
+    for (int h = 0; h < H; ++h)
+      if (mine[h]) tslot[h] = rank * text_slots + used++;
+    if (mine[H - 1]) tslot[H] = rank * text_slots + used++;
+  }
+  std::vector<int> own_scored, xrow0(std::max(H - 1, 1), 0);
+  for (int h = 0; h + 1 < H; ++h) {
+    if (!passing) break;
+    xrow0[h] = (owner[h] * pass_slots + pslot[h]) * p->P;
+    if (mine[h]) own_scored.push_back(h);
+  }
+  const auto local = build_local_items(*p, &mine, &tslot);
+  const auto remote = build_remote_items(*p, &mine);
+  const auto probe = build_probe_items(*p, H - 1, &mine);
+  const auto score = passing ? build_score_items(*p, H - 1, &mine) : std::vector<int4>();
+  TablePacker tab;
+  const size_t o_hosts = tab.put(own_scored.data(), own_scored.size() * 4);
+  const size_t o_xrow = tab.put(xrow0.data(), xrow0.size() * 4);
+  const size_t o_score = tab.put(score.data(), score.size() * sizeof(int4));
+  const size_t o_local = tab.put(local.data(), local.size() * sizeof(AttnItem));
+  const size_t o_remote = tab.put(remote.data(), remote.size() * sizeof(AttnItem));
+  const size_t o_probe = tab.put(probe.data(), probe.size() * sizeof(AttnItem));
+  if (p->dtab_shard) {
+    SPAVA_CUDA(cudaDeviceSynchronize());
+    SPAVA_CUDA(cudaFree(p->dtab_shard));
+    p->dtab_shard = nullptr;
+    p->shard_world = 0;
+  }
+  void* d = nullptr;
+  spava_status st = upload_table(tab.host, &d);
+  if (st != SPAVA_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(d);
+  p->dtab_shard = d;
+  p->shard_rank = rank;
+  p->shard_world = world;
+  p->owner.assign(owner, owner + H);
+  p->pass_slots = pass_slots;
+  p->text_slots = text_slots;
+  p->text_slots_used = used;
+  p->d_shard_hosts = reinterpret_cast<int*>(base + o_hosts);
+  p->n_shard_hosts = static_cast<int>(own_scored.size());
+  p->d_xrow0 = reinterpret_cast<int*>(base + o_xrow);
+  p->d_score_shard = reinterpret_cast<int4*>(base + o_score);
+  p->n_score_shard = static_cast<int>(score.size());
+  p->d_items_shard_local = reinterpret_cast<AttnItem*>(base + o_local);
+  p->n_items_shard_local = static_cast<int>(local.size());
+  p->d_items_shard_remote = reinterpret_cast<AttnItem*>(base + o_remote);
+  p->n_items_shard_remote = static_cast<int>(remote.size());
+  p->d_items_shard_probe = reinterpret_cast<AttnItem*>(base + o_probe);
+  p->n_items_shard_probe = static_cast<int>(probe.size());
+  layout_workspace(p);
+  return ok();
+}
+
+spava_status spava_shard_query(const spava_plan* p, spava_shard_layout* out) {
+  if (!p || !out) return fail(SPAVA_ERR_INVALID_ARG, "plan and out must not be NULL");
+  if (p->shard_world == 0) return fail(SPAVA_ERR_INVALID_ARG, "plan is not sharded (spava_plan_set_shard)");
+  spava_shard_layout l;
+  std::memset(&l, 0, sizeof(l));
+  l.workspace_bytes = p->ws_total_shard;
+  l.pass_k_offset = p->ws_xk;
+  l.pass_v_offset = p->ws_xv;
+  l.pass_bytes_per_rank = static_cast<uint64_t>(p->pass_slots) * p->P * score_rows(*p) * p->d * 2;
+  l.text_o_offset = p->ws_to;
+  l.text_o_bytes_per_rank = static_cast<uint64_t>(p->text_slots) * p->T * p->hq * p->d * 4;
+  l.text_lse_offset = p->ws_tl;
+  l.text_lse_bytes_per_rank = static_cast<uint64_t>(p->text_slots) * p->hq * p->T * 4;
+  l.scores_offset = p->ws_scores;
+  l.idx_offset = p->ws_idx;
+  l.pass_slots = p->pass_slots;
+  l.text_slots = p->text_slots;
+  *out = l;
+  return ok();
+}
+
+spava_status spava_shard_stage(const spava_plan* p, int32_t stage, const void* q, const void* k, const void* v,
+                               void* o, float* lse, void* ws, void* stream) {
+  spava_status s;
+  if ((s = check_plan_ws(p, ws)) != SPAVA_OK) return s;
+  if (p->shard_world == 0) return fail(SPAVA_ERR_INVALID_ARG, "plan is not sharded (spava_plan_set_shard)");
+  if (stage < SPAVA_SHARD_SELECT || stage > SPAVA_SHARD_MERGE) return fail(SPAVA_ERR_INVALID_ARG, "unknown stage %d", stage);
+  const bool need_qkv = stage != SPAVA_SHARD_MERGE, need_o = stage != SPAVA_SHARD_SELECT;
+  if (need_qkv && (!q || !k || !v)) return fail(SPAVA_ERR_INVALID_ARG, "NULL q, k or v");
+  if (need_o && (!o || !lse)) return fail(SPAVA_ERR_INVALID_ARG, "NULL o or lse");
+  if ((need_qkv && (!aligned16(q) || !aligned16(k) || !aligned16(v))) || (need_o && !aligned16(o)))
+    return fail(SPAVA_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = begin_call(p, ws, st, stage == SPAVA_SHARD_SELECT)) != SPAVA_OK) return s;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  TwoStageBufs ts;
+  ts.row_o = reinterpret_cast<float*>(w + p->ws_row_o);
+  ts.row_lse = reinterpret_cast<float*>(w + p->ws_row_lse);
+  ts.text_o = reinterpret_cast<float*>(w + p->ws_to);
+  ts.text_lse = reinterpret_cast<float*>(w + p->ws_tl);
+  const size_t pass_part = static_cast<size_t>(p->pass_slots) * p->P * score_rows(*p) * p->d * 2;
+  switch (stage) {
+    case SPAVA_SHARD_SELECT: {
+      if (!scores_needed(*p) || p->n_shard_hosts == 0) break;
+      float* scores = reinterpret_cast<float*>(w + p->ws_scores);
+      int32_t* idx = reinterpret_cast<int32_t*>(w + p->ws_idx);
+      if ((s = launch_probe_lse(p, q, k, k, ws, st, p->d_items_shard_probe, p->n_items_shard_probe)) != SPAVA_OK)
+        return s;
+      s = p->d == 128 ? launch_score<128>(p, q, k, scores, p->d_score_shard, p->n_score_shard, ws, st)
+                      : launch_score<64>(p, q, k, scores, p->d_score_shard, p->n_score_shard, ws, st);
+      if (s != SPAVA_OK) return s;
+      PassDest dst{w + p->ws_xk + p->shard_rank * pass_part, w + p->ws_xv + p->shard_rank * pass_part, true};
+      if ((s = launch_select(p, scores, idx, st, k, v, dst, p->d_shard_hosts, p->n_shard_hosts)) != SPAVA_OK) return s;
+      break;
+    }
+    case SPAVA_SHARD_LOCAL: {
+      const int spare = p->text_slots - p->text_slots_used;
+      if (p->T > 0 && spare > 0) {  // this rank's unused text slots: O = 0, lse = -inf
+        const size_t slot0 = static_cast<size_t>(p->shard_rank) * p->text_slots + p->text_slots_used;
+        const size_t n_o = static_cast<size_t>(spare) * p->T * p->hq * p->d, n_l = static_cast<size_t>(spare) * p->hq * p->T;
+        uint32_t* fo = reinterpret_cast<uint32_t*>(ts.text_o) + slot0 * p->T * p->hq * p->d;
+        uint32_t* fl = reinterpret_cast<uint32_t*>(ts.text_lse) + slot0 * p->hq * p->T;
+        const int grid = std::max(1, std::min(p->num_sms * 4, static_cast<int>((n_o + 255) / 256)));
+        mark(p, kLabFill, st);
+        spava::fill_u32_kernel<<<grid, 256, 0, st>>>(fo, n_o, 0u);
+        spava::fill_u32_kernel<<<grid, 256, 0, st>>>(fl, n_l, 0xFF800000u);
+        SPAVA_CUDA(cudaGetLastError());
+        g_last_launches += 2;
+      }
+      s = p->d == 128 ? launch_attn<128>(p, p->d_items_shard_local, p->n_items_shard_local, q, k, v, nullptr, nullptr,
+                                         o, lse, ws, st, ts)
+                      : launch_attn<64>(p, p->d_items_shard_local, p->n_items_shard_local, q, k, v, nullptr, nullptr,
+                                        o, lse, ws, st, ts);
+      if (s != SPAVA_OK) return s;
+      break;
+    }
+    case SPAVA_SHARD_REMOTE: {
+      if (p->n_items_shard_remote == 0) break;
+      void* kp = w + p->ws_kp;
+      void* vp = w + p->ws_vp;
+      if (scores_needed(*p)) {
+        const int rows = score_rows(*p), cpr = p->d * 2 / 16;
+        const size_t total = static_cast<size_t>(rows) * (p->H - 1) * p->P * cpr;
+        const int grid = static_cast<int>(std::min<size_t>((total + 255) / 256, static_cast<size_t>(p->num_sms) * 8));
+        mark(p, kLabUnpack, st);
+        spava::unpack_passing_kernel<<<grid, 256, 0, st>>>(
+            reinterpret_cast<const uint4*>(w + p->ws_xk), reinterpret_cast<const uint4*>(w + p->ws_xv), p->d_xrow0,
+            static_cast<uint4*>(kp), static_cast<uint4*>(vp), rows, p->H - 1, p->P, cpr);
+        SPAVA_CUDA(cudaGetLastError());
+        ++g_last_launches;
+      }
+      s = p->d == 128 ? launch_attn<128>(p, p->d_items_shard_remote, p->n_items_shard_remote, q, k, v, kp, vp, o, lse,
+                                         ws, st, ts)
+                      : launch_attn<64>(p, p->d_items_shard_remote, p->n_items_shard_remote, q, k, v, kp, vp, o, lse,
+                                        ws, st, ts);
+      if (s != SPAVA_OK) return s;
+      break;
+    }
+    case SPAVA_SHARD_MERGE: {
+      if ((s = launch_merge(p, o, lse, ws, st, ts.text_o, ts.text_lse, p->shard_world * p->text_slots)) != SPAVA_OK)
+        return s;
+      break;
+    }
+  }
   mark(p, -1, st);
   return ok();
 }
@@ -1023,6 +1336,7 @@ const char* spava_kernel_name(int32_t label) {
     case kLabAttnLocal: return "attention_local";
     case kLabAttnRemote: return "attention_remote";
     case kLabProbeLse: return "probe_lse";
+    case kLabUnpack: return "unpack_passing";
   }
   return "unknown";
 }

@@ -502,3 +502,60 @@ def test_frame_structure():
     f0 = plain[plain < 64]
     spread = np.abs(k[f0, 0] - k[f0, 0].mean(axis=0)).mean()
     assert 0.15 < spread < 0.35
+
+
+# ---------------------------------------------------------------- sharding (multi-host form)
+def test_zigzag_pages_example():
+    """The pages' description of the arrangement (German explainer, "Lastverteilung"):
+    the first worker takes the first and the last block, the second the second and the
+    one before last, and so on -- here 4 workers and 8 blocks, and 1 worker and 2."""
+    assert orc.zigzag_owners(8, 4).tolist() == [0, 1, 2, 3, 3, 2, 1, 0]
+    assert orc.zigzag_owners(2, 1).tolist() == [0, 0]
+    with pytest.raises(ValueError):
+        orc.zigzag_owners(6, 4)
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("rounds", [1, 2, 3])
+def test_zigzag_balances_passing_lengths(world, rounds):
+    """"Approximate attention load balancing": ZigZag makes the total length of the
+    passing blocks each physical host attends to equal (host h attends to h * P passing
+    rows); every rank runs the same number of hosts.  The contiguous split does not
+    balance (later ranks carry more) once there are two ranks."""
+    H, P = 2 * world * rounds, 7
+    zz = orc.zigzag_owners(H, world)
+    load = np.zeros(world, dtype=np.int64)
+    for h in range(H):
+        load[zz[h]] += h * P
+    assert (load == load[0]).all()
+    assert (np.bincount(zz, minlength=world) == 2 * rounds).all()
+    ct = orc.contiguous_owners(H, world)
+    lc = np.zeros(world, dtype=np.int64)
+    for h in range(H):
+        lc[ct[h]] += h * P
+    assert (world == 1) or (np.diff(lc) > 0).all()
+
+
+@pytest.mark.parametrize("policy", ["zigzag", "contiguous", "random"])
+@pytest.mark.parametrize("head_reduce", ["max", "none"])
+def test_sharded_attention_equals_single(policy, head_reduce):
+    """The multi-host form (local causal part and [anchor | passing] part merged
+    through the lse per host; the text rows' per-host partials from their owners,
+    merged after the exchange) equals the one-pass approximate attention."""
+    H, world = 8, 2
+    cfg = CONFIGS["tiny"].with_(n_visual=256, n_hosts=H, n_text=11, hq=4, hkv=2, head_dim=16, anchor=8,
+                                passing=5, probe_r=16)
+    g = generate(cfg)
+    q, k, v = (orc.bf16_bits_to_f64(g[x]) for x in ("q", "k", "v"))
+    scale = 1 / math.sqrt(cfg.head_dim)
+    res = orc.prefill(q, k, v, g["host_sizes"], cfg.anchor, cfg.passing, cfg.probe_r, scale=scale,
+                      head_reduce=head_reduce)
+    if policy == "zigzag":
+        owner = orc.zigzag_owners(H, world)
+    elif policy == "contiguous":
+        owner = orc.contiguous_owners(H, world)
+    else:
+        owner = np.random.default_rng(5).integers(0, 3, size=H)
+    O, L = orc.sharded_attention(q, k, v, res["offsets"], cfg.anchor, res["sel"], scale, owner)
+    np.testing.assert_allclose(O, res["O"], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(L, res["lse"], rtol=1e-12, atol=1e-12)
