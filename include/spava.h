@@ -344,7 +344,9 @@ spava_status spava_shard_query(const spava_plan* plan, spava_shard_layout* out);
  *   SPAVA_SHARD_MERGE   text rows from all ranks' text slots (needs the gathered
  *                       text_o / text_lse): final O/lse of rows [N, N+T).
  * q, k, v, o [N+T][heads][d] bf16 and lse [hq][N+T] are full-size device buffers with
- * the layouts above; rows a rank does not own are neither read nor written.  `ws`
+ * the layouts above.  Rows a rank does not own are not written and do not change the
+ * result, but they must hold finite values (zeros will do): a 128-row tile can load
+ * rows past the end of a block, which then take part with weight exactly 0.  `ws`
  * holds spava_shard_layout.workspace_bytes.  Together the four stages over all
  * ranks compute spava_attn_prefill_two_stage's result with the score kernel's
  * scores (spava_attn_prefill's selection). */

@@ -49,7 +49,7 @@ Readings taken where they are silent (each is a parameter of this oracle):
   R7  ties in selection: larger score first; equal scores -> lower token index;
       -0.0 equals +0.0.  The P chosen indices are stored in ascending order.
   R8  GQA: query head c uses KV head c // (hq / hkv) (parity unpinned).
-  R9  ZigZag arrangement with more than 2W virtual hosts on W ranks: the pairing of
+  R11 ZigZag arrangement with more than 2W virtual hosts on W ranks: the pairing of
       rank r with virtual hosts r and 2W-1-r repeats over consecutive rounds of 2W
       hosts (the pages only describe one round).
 """
@@ -326,7 +326,7 @@ def zigzag_owners(n_hosts: int, world: int) -> np.ndarray:
     splitting & ZigZag arrangement": a physical host runs the pair of virtual hosts h
     and 2H-1-h; the German explainer, "Lastverteilung": the first worker takes the
     first and the last block, the second the second and the one before last, and so
-    on).  Rank of each of n_hosts virtual hosts on ``world`` ranks; reading R9 for
+    on).  Rank of each of n_hosts virtual hosts on ``world`` ranks; reading R11 for
     n_hosts > 2 * world."""
     if world < 1 or n_hosts % (2 * world):
         raise ValueError("zigzag needs n_hosts to be a multiple of 2 * world")

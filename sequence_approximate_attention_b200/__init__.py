@@ -97,8 +97,7 @@ class Plan:
             raise ValueError(f"score reduction must be one of {sorted(self.SCORE_REDUCE)}")
         _lib.check(self.lib.spava_plan_set_score_reduce(self._h, self.SCORE_REDUCE[mode]), "spava_plan_set_score_reduce")
         self.score_reduce = mode
-        self.workspace_bytes = int(self.lib.spava_workspace_bytes(self._h))
-        self.two_stage_workspace_bytes = int(self.lib.spava_two_stage_workspace_bytes(self._h))
+        self._refresh_sizes()
 
     SCORE_KIND = {"logit": 0, "prob": 1}
 
@@ -109,8 +108,13 @@ class Plan:
             raise ValueError(f"score kind must be one of {sorted(self.SCORE_KIND)}")
         _lib.check(self.lib.spava_plan_set_score_kind(self._h, self.SCORE_KIND[kind]), "spava_plan_set_score_kind")
         self.score_kind = kind
+        self._refresh_sizes()
+
+    def _refresh_sizes(self) -> None:
         self.workspace_bytes = int(self.lib.spava_workspace_bytes(self._h))
         self.two_stage_workspace_bytes = int(self.lib.spava_two_stage_workspace_bytes(self._h))
+        if getattr(self, "shard_world", 0):
+            self.shard_workspace_bytes = int(self.shard_layout().workspace_bytes)
 
     def set_shard(self, rank: int, world: int, owner: Sequence[int]) -> None:
         """spava_plan_set_shard: this plan runs rank ``rank`` of ``world``, host h on rank
@@ -121,6 +125,7 @@ class Plan:
         with torch.cuda.device(self.device):
             _lib.check(self.lib.spava_plan_set_shard(self._h, int(rank), int(world), arr), "spava_plan_set_shard")
         self.shard_rank, self.shard_world, self.owner = int(rank), int(world), [int(x) for x in owner]
+        self._refresh_sizes()
 
     def shard_layout(self) -> "_lib.ShardLayout":
         """spava_shard_query: byte offsets of the exchange buffers in the sharded workspace."""
@@ -340,7 +345,9 @@ def shard_stage(plan: Plan, stage: int, q: Optional[torch.Tensor], k: Optional[t
     if stage != _lib.SPAVA_SHARD_SELECT:
         _expect(o, "o", torch.bfloat16, (plan.n_total, plan.hq, plan.head_dim), dev)
         _expect(lse, "lse", torch.float32, (plan.hq, plan.n_total), dev)
-    need = int(plan.shard_layout().workspace_bytes)
+    need = getattr(plan, "shard_workspace_bytes", None)
+    if need is None:
+        raise ValueError("plan is not sharded (Plan.set_shard)")
     if workspace.dtype != torch.uint8 or workspace.numel() < need or workspace.device != dev or \
             workspace.data_ptr() % 256:
         raise ValueError(f"workspace: uint8, 256-byte aligned, >= {need} bytes on the plan's device")

@@ -94,7 +94,8 @@ class ShardedPrefill:
                 lse: Optional[torch.Tensor] = None):
         """One layer on this rank.  q/k/v are full-size [N+T, heads, d] buffers holding
         this rank's host rows and the text rows (the anchor rows arrive by broadcast);
-        returns (o, lse) with this rank's host rows and all text rows final."""
+        their other rows must be finite (zeros will do).  Returns (o, lse) with this
+        rank's host rows and all text rows final."""
         plan = self.plan
         if o is None:
             o = torch.empty_like(q)

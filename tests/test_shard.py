@@ -150,7 +150,7 @@ def _rank_main(rank, world, port, owner, out):
 @pytest.mark.parametrize("owner", [[0, 1, 1, 0], [1, 0, 0, 1], [0, 0, 1, 1]])
 def test_sharded_orchestration_two_gloo_ranks(owner):
     world = 2
-    with mp.Manager() as man:
+    with mp.get_context("spawn").Manager() as man:
         out = man.dict()
         mp.spawn(_rank_main, args=(world, _free_port(), owner, out), nprocs=world, join=True)
         res = dict(out)
