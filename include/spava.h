@@ -282,14 +282,38 @@ spava_status spava_dense_causal(const spava_plan* plan, const void* q, const voi
  *   SPAVA_SHARD_ZIGZAG      the hosts form rounds of 2*world; in each round rank r runs
  *                           hosts r and 2*world-1-r (a later host attends to more
  *                           passing rows, so the pairs carry equal passing lengths).
+ *   SPAVA_SHARD_LONGEST_FIRST  (spava_plan_shard_owners only) hosts by decreasing
+ *                           cost, each to the rank with the least cost so far (ties to
+ *                           the lower host, then the lower rank); a host's cost is the
+ *                           (query, key) pairs its rows and its text piece attend:
+ *                           B(B+1)/2 + B(A + hP) for h >= 1, + T B, and T(T+1)/2 more
+ *                           for the last host (the text rows' causal part).  The one-GPU
+ *                           scheduler's longest-first rule applied to whole hosts; it
+ *                           balances uneven blocks, which the pairing does not.
  */
-typedef enum { SPAVA_SHARD_CONTIGUOUS = 0, SPAVA_SHARD_ZIGZAG = 1 } spava_shard_policy;
+typedef enum {
+  SPAVA_SHARD_CONTIGUOUS = 0,
+  SPAVA_SHARD_ZIGZAG = 1,
+  SPAVA_SHARD_LONGEST_FIRST = 2
+} spava_shard_policy;
 
 /* Host-side only (no device needed): owner_out[h] = the rank that runs host h, for a
  * HOST array of n_hosts ints.  CONTIGUOUS needs n_hosts % world == 0, ZIGZAG
  * n_hosts % (2 * world) == 0; otherwise, or for a NULL array or world < 1, returns
  * SPAVA_ERR_INVALID_ARG and writes nothing. */
 spava_status spava_shard_owners(int32_t n_hosts, int32_t world, int32_t policy, int32_t* owner_out);
+
+/* Longest-first assignment of n_hosts hosts with the given costs (HOST array of
+ * n_hosts int64 >= 0) to `world` ranks, into owner_out (HOST array).  Host-side only.
+ * SPAVA_ERR_INVALID_ARG for NULL arrays, n_hosts < 1, world < 1 or a negative cost. */
+spava_status spava_shard_owners_by_cost(int32_t n_hosts, int32_t world, const int64_t* cost,
+                                        int32_t* owner_out);
+
+/* Ownership for this plan's host sizes: CONTIGUOUS and ZIGZAG as spava_shard_owners,
+ * LONGEST_FIRST from the plan's per-host costs above (any H >= 1, world >= 1).
+ * Host-side only; owner_out is a HOST array of H ints.  SPAVA_ERR_INVALID_ARG as
+ * above. */
+spava_status spava_plan_shard_owners(const spava_plan* plan, int32_t world, int32_t policy, int32_t* owner_out);
 
 /* Make `plan` run rank `rank` of `world`, host h on rank owner[h] (HOST array of H
  * ints in [0, world), copied; every rank of a job passes the same array).  Builds this

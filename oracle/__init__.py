@@ -13,9 +13,11 @@ from .spava_oracle import (  # noqa: F401
     bf16_bits_to_f64,
     contiguous_owners,
     dense_causal,
+    host_costs,
     host_of_row,
     host_offsets,
     key_set,
+    longest_first_owners,
     lse_merge,
     prefill,
     probe_scores,

@@ -396,3 +396,35 @@ def sharded_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, off: np.ndarr
                 o_t, l_t = lse_merge(o_t, l_t, op, lp)
             O[N:NT, c], lse[c, N:NT] = o_t, l_t
     return O, lse
+
+
+def host_costs(host_sizes: Sequence[int], anchor: int, passing: int, n_text: int) -> np.ndarray:
+    """Work of each host in (query, key) pairs: its rows over its own block (causal),
+    over the anchor and the passing rows of the earlier hosts (h >= 1), and the text
+    rows over its block; the last host also carries the text rows' causal part (the
+    piece that sharding puts on its rank).  Summed over the hosts this is the number
+    of pairs the whole approximate attention evaluates per query head."""
+    H = len(host_sizes)
+    cost = np.zeros(H, dtype=np.int64)
+    for h, B in enumerate(int(b) for b in host_sizes):
+        cost[h] = B * (B + 1) // 2 + n_text * B
+        if h >= 1:
+            cost[h] += B * (anchor + h * passing)
+        if h == H - 1:
+            cost[h] += n_text * (n_text + 1) // 2
+    return cost
+
+
+def longest_first_owners(cost: Sequence[int], world: int) -> np.ndarray:
+    """Longest-processing-time list scheduling: hosts taken by decreasing cost (equal
+    costs in host order), each given to the rank with the least cost so far (the
+    lowest such rank).  The one-GPU scheduler's longest-first rule applied to whole
+    hosts across ranks."""
+    order = sorted(range(len(cost)), key=lambda h: (-int(cost[h]), h))
+    load = [0] * world
+    owner = np.empty(len(cost), dtype=np.int64)
+    for h in order:
+        r = min(range(world), key=lambda x: (load[x], x))
+        owner[h] = r
+        load[r] += int(cost[h])
+    return owner

@@ -127,6 +127,16 @@ class Plan:
         self.shard_rank, self.shard_world, self.owner = int(rank), int(world), [int(x) for x in owner]
         self._refresh_sizes()
 
+    def shard_owners(self, world: int, policy: str = "zigzag"):
+        """spava_plan_shard_owners: the rank of every host; "longest_first" balances this
+        plan's per-host costs (uneven blocks), the others as shard_owners()."""
+        if policy not in SHARD_POLICY:
+            raise ValueError(f"policy must be one of {sorted(SHARD_POLICY)}")
+        arr = (ctypes.c_int32 * self.n_hosts)()
+        _lib.check(self.lib.spava_plan_shard_owners(self._h, int(world), SHARD_POLICY[policy], arr),
+                   "spava_plan_shard_owners")
+        return [int(x) for x in arr]
+
     def shard_layout(self) -> "_lib.ShardLayout":
         """spava_shard_query: byte offsets of the exchange buffers in the sharded workspace."""
         out = _lib.ShardLayout()
@@ -319,12 +329,13 @@ def dense_causal(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return o, lse
 
 
-SHARD_POLICY = {"contiguous": _lib.SPAVA_SHARD_CONTIGUOUS, "zigzag": _lib.SPAVA_SHARD_ZIGZAG}
+SHARD_POLICY = {"contiguous": _lib.SPAVA_SHARD_CONTIGUOUS, "zigzag": _lib.SPAVA_SHARD_ZIGZAG,
+                "longest_first": _lib.SPAVA_SHARD_LONGEST_FIRST}
 
 
 def shard_owners(n_hosts: int, world: int, policy: str = "zigzag"):
     """spava_shard_owners (host-side, no device): the rank of every host under the
-    "contiguous" or "zigzag" policy."""
+    "contiguous" or "zigzag" policy ("longest_first" needs the plan: Plan.shard_owners)."""
     if policy not in SHARD_POLICY:
         raise ValueError(f"policy must be one of {sorted(SHARD_POLICY)}")
     lib = _lib.load()

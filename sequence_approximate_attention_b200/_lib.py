@@ -18,6 +18,7 @@ SPAVA_SCORES_GIVEN = 1
 
 SPAVA_SHARD_CONTIGUOUS = 0
 SPAVA_SHARD_ZIGZAG = 1
+SPAVA_SHARD_LONGEST_FIRST = 2
 SPAVA_SHARD_SELECT, SPAVA_SHARD_LOCAL, SPAVA_SHARD_REMOTE, SPAVA_SHARD_MERGE = 0, 1, 2, 3
 
 
@@ -55,6 +56,9 @@ SIGNATURES = {
     "spava_dense_causal": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                      c_void_p, c_void_p, c_void_p]),
     "spava_shard_owners": (c_int32, [c_int32, c_int32, c_int32, ctypes.POINTER(c_int32)]),
+    "spava_shard_owners_by_cost": (c_int32, [c_int32, c_int32, ctypes.POINTER(ctypes.c_int64),
+                                             ctypes.POINTER(c_int32)]),
+    "spava_plan_shard_owners": (c_int32, [c_void_p, c_int32, c_int32, ctypes.POINTER(c_int32)]),
     "spava_plan_set_shard": (c_int32, [c_void_p, c_int32, c_int32, ctypes.POINTER(c_int32)]),
     "spava_shard_query": (c_int32, [c_void_p, ctypes.POINTER(ShardLayout)]),
     "spava_shard_stage": (c_int32, [c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,

@@ -1102,6 +1102,39 @@ spava_status spava_shard_owners(int32_t n_hosts, int32_t world, int32_t policy, 
   return fail(SPAVA_ERR_INVALID_ARG, "unknown shard policy %d", policy);
 }
 
+spava_status spava_plan_shard_owners(const spava_plan* p, int32_t world, int32_t policy, int32_t* owner_out) {
+  if (!p || !owner_out || world < 1) return fail(SPAVA_ERR_INVALID_ARG, "need a plan, world >= 1 and an array");
+  if (policy != SPAVA_SHARD_LONGEST_FIRST) return spava_shard_owners(p->H, world, policy, owner_out);
+  const int H = p->H;
+  std::vector<int64_t> cost(H);
+  for (int h = 0; h < H; ++h) {
+    const int64_t B = p->off[h + 1] - p->off[h];
+    cost[h] = B * (B + 1) / 2 + static_cast<int64_t>(p->T) * B;
+    if (h >= 1) cost[h] += B * (p->A + static_cast<int64_t>(h) * p->P);
+    if (h == H - 1) cost[h] += static_cast<int64_t>(p->T) * (p->T + 1) / 2;
+  }
+  return spava_shard_owners_by_cost(H, world, cost.data(), owner_out);
+}
+
+spava_status spava_shard_owners_by_cost(int32_t n_hosts, int32_t world, const int64_t* cost, int32_t* owner_out) {
+  if (!cost || !owner_out || n_hosts < 1 || world < 1)
+    return fail(SPAVA_ERR_INVALID_ARG, "need H >= 1, world >= 1 and two arrays");
+  for (int h = 0; h < n_hosts; ++h)
+    if (cost[h] < 0) return fail(SPAVA_ERR_INVALID_ARG, "host %d has a negative cost", h);
+  std::vector<int> order(n_hosts);
+  for (int h = 0; h < n_hosts; ++h) order[h] = h;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+  std::vector<int64_t> load(world, 0);
+  for (int h : order) {
+    int best = 0;
+    for (int r = 1; r < world; ++r)
+      if (load[r] < load[best]) best = r;
+    owner_out[h] = best;
+    load[best] += cost[h];
+  }
+  return ok();
+}
+
 spava_status spava_plan_set_shard(spava_plan* p, int32_t rank, int32_t world, const int32_t* owner) {
   if (!p || !owner) return fail(SPAVA_ERR_INVALID_ARG, "plan and owner must not be NULL");
   if (world < 1 || rank < 0 || rank >= world) return fail(SPAVA_ERR_INVALID_ARG, "need 0 <= rank < world");

@@ -1,7 +1,7 @@
 """Per-rank compute of the sharded prefill, measured on one GPU.
 
     python -m sequence_approximate_attention_b200.shard_emulate --config 128k \\
-        --worlds 2,4,8 --policies zigzag,contiguous
+        --worlds 2,4,8 --policies zigzag,contiguous,longest_first
 
 For each (world W, ownership policy) it builds the W ranks' plans on this GPU, runs
 their stages in the order a W-GPU job would (every rank's SELECT, the exchange, every
@@ -26,7 +26,7 @@ import sys
 import numpy as np
 import torch
 
-from . import Plan, _lib, attn_prefill, shard_owners, shard_stage
+from . import Plan, _lib, attn_prefill, shard_stage
 
 STAGES = (_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_LOCAL, _lib.SPAVA_SHARD_REMOTE, _lib.SPAVA_SHARD_MERGE)
 STAGE_NAMES = ("select", "local", "remote", "merge")
@@ -50,7 +50,9 @@ def _plan(cfg, sizes, dev):
 
 def emulate(cfg, sizes, q, k, v, world, policy, steps, warmup):
     dev = q.device
-    owner = shard_owners(cfg.n_hosts, world, policy)
+    probe = _plan(cfg, sizes, dev)
+    owner = probe.shard_owners(world, policy)
+    probe.close()
     ranks = []
     for r in range(world):
         p = _plan(cfg, sizes, dev)
@@ -130,7 +132,7 @@ def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--config", default="128k", choices=sorted(CONFIGS))
     ap.add_argument("--worlds", default="2,4,8")
-    ap.add_argument("--policies", default="zigzag,contiguous")
+    ap.add_argument("--policies", default="zigzag,contiguous,longest_first")
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     args = ap.parse_args(argv)

@@ -248,3 +248,68 @@ def test_fullsize_score_variants_qwen64k(reduce, kind):
     plan.close()
     del dev, o, lse, ws
     torch.cuda.empty_cache()
+
+
+def test_fullsize_sharded_emulated(fullsize_run):
+    """The sharded prefill at full size, its W ranks run one after another on this GPU
+    (128k: W = 8, ZigZag; stress: W = 4, ZigZag, uneven blocks), the exchange moved by
+    device copies between the stages: every host's selection equals the one-GPU
+    prefill's bit for bit; O and lse of every row within the bf16 tolerances of the
+    one-GPU prefill's; sampled outputs against the oracle."""
+    r = fullsize_run
+    cfg = r["cfg"]
+    worlds = {"128k": 8, "stress": 4}
+    if cfg.name not in worlds:
+        pytest.skip("sharded prefill checked at full size on the 128k and stress workloads")
+    W, dev = worlds[cfg.name], r["dev"]
+    owner = sab.shard_owners(cfg.n_hosts, W, "zigzag")
+    ranks = []
+    for rk in range(W):
+        p = sab.Plan(cfg.n_visual, cfg.n_text, cfg.n_hosts, r["sizes"], cfg.anchor, cfg.passing, cfg.probe_r,
+                     cfg.hq, cfg.hkv, cfg.head_dim)
+        p.set_shard(rk, W, owner)
+        ranks.append((p, p.shard_layout(), torch.zeros(p.shard_workspace_bytes, dtype=torch.uint8, device="cuda")))
+    o = torch.zeros_like(dev["q"])
+    lse = torch.zeros_like(r["lse"])
+    L0 = ranks[0][1]
+
+    def exchange(off, per):
+        off, per = int(off), int(per)
+        for rk, (_, _, ws) in enumerate(ranks):
+            for _, _, ws2 in ranks:
+                if ws2 is not ws:
+                    ws2[off + rk * per: off + (rk + 1) * per].copy_(ws[off + rk * per: off + (rk + 1) * per])
+
+    from sequence_approximate_attention_b200 import _lib
+    for sid in (_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_LOCAL, _lib.SPAVA_SHARD_REMOTE, _lib.SPAVA_SHARD_MERGE):
+        for p, _, ws in ranks:
+            sab.shard_stage(p, sid, dev["q"], dev["k"], dev["v"], o, lse, ws)
+        if sid == _lib.SPAVA_SHARD_SELECT:
+            exchange(L0.pass_k_offset, L0.pass_bytes_per_rank)
+            exchange(L0.pass_v_offset, L0.pass_bytes_per_rank)
+        elif sid == _lib.SPAVA_SHARD_LOCAL:
+            exchange(L0.text_o_offset, L0.text_o_bytes_per_rank)
+            exchange(L0.text_lse_offset, L0.text_lse_bytes_per_rank)
+    for p, _, ws in ranks:
+        sab.check_device_error(p, ws)
+    H, P, hkv = cfg.n_hosts, cfg.passing, cfg.hkv
+    sel = np.empty_like(r["idx"])
+    for h in range(H - 1):
+        p, L, ws = ranks[owner[h]]
+        idx = ws[int(L.idx_offset): int(L.idx_offset) + (H - 1) * hkv * P * 4].view(torch.int32).view(H - 1, hkv, P)
+        sel[h] = idx[h].cpu().numpy()
+    np.testing.assert_array_equal(sel, r["idx"])
+    do = (o.float() - r["o"].float()).abs().max().item()
+    dl = (lse - r["lse"]).abs().max().item()
+    assert do <= O_TOL and dl <= LSE_TOL, (cfg.name, do, dl)
+    off = orc.host_offsets(r["sizes"])
+    q, k, v = (LazyF64(r["g"][x]) for x in ("q", "k", "v"))
+    rows, heads = _sample_rows(cfg, off, np.random.default_rng(cfg.seed + 2))
+    O_ref, L_ref = orc.attention_rows(q, k, v, off, cfg.anchor, sel, 1.0 / math.sqrt(cfg.head_dim), rows, heads)
+    rt, ht = torch.tensor(rows, device="cuda"), torch.tensor(heads, device="cuda")
+    assert np.abs(o[rt, ht].float().cpu().numpy() - O_ref).max() <= O_TOL
+    assert np.abs(lse[ht, rt].cpu().numpy() - L_ref).max() <= LSE_TOL
+    for p, _, _ in ranks:
+        p.close()
+    del ranks, o, lse
+    torch.cuda.empty_cache()

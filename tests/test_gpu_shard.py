@@ -48,7 +48,18 @@ CASES = {
     "prob_w2": (BASE, None, [0, 1, 1, 0], "max", "prob"),
     "one_host": (BASE.with_(n_hosts=1), None, [0], "max", "logit"),
     "no_anchor_no_passing_w2": (BASE.with_(anchor=0, passing=0), None, [0, 1, 1, 0], "max", "logit"),
+    # owners from the oracle's longest-first rule on these uneven blocks (3 ranks)
+    "longest_first_w3_uneven": (BASE.with_(n_hosts=8, head_dim=64, anchor=16, passing=48),
+                                [96, 160, 128, 112, 144, 128, 100, 156], "longest_first:3", "max", "logit"),
 }
+
+
+def _owner(cfg, sizes, owner):
+    if isinstance(owner, str):
+        world = int(owner.split(":")[1])
+        cost = orc.host_costs(sizes, cfg.anchor, cfg.passing, cfg.n_text)
+        return orc.longest_first_owners(cost, world).tolist()
+    return owner
 
 
 def _garbage_like(t, rng_seed):
@@ -62,6 +73,7 @@ def _run_emulated(name):
     g, f64, dev = inputs(cfg)
     sizes = np.asarray(sizes if sizes is not None else g["host_sizes"], dtype=np.int32)
     off = orc.host_offsets(sizes)
+    owner = _owner(cfg, sizes, owner)
     H, N, NT, A = cfg.n_hosts, cfg.n_visual, cfg.n_total, cfg.anchor
     world = max(owner) + 1
     ranks = []
@@ -184,4 +196,21 @@ def test_stage_needs_a_shard():
                                       ws.data_ptr(), None) == _lib.SPAVA_ERR_INVALID_ARG
     assert plan.lib.spava_shard_stage(plan.handle, _lib.SPAVA_SHARD_LOCAL, None, None, None, None, None,
                                       ws.data_ptr(), None) == _lib.SPAVA_ERR_INVALID_ARG
+    plan.close()
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 5])
+def test_plan_owners_match_oracle(world):
+    """spava_plan_shard_owners: longest first from the plan's per-host costs (uneven
+    blocks, text rows) equals the oracle's rule on its host_costs; the pairing policies
+    equal spava_shard_owners'."""
+    cfg = BASE.with_(n_hosts=8, head_dim=64, anchor=16, passing=48, n_text=70)
+    sizes = [96, 160, 128, 112, 144, 128, 100, 156]
+    plan = make_plan(sab, cfg, sizes)
+    want = orc.longest_first_owners(orc.host_costs(sizes, cfg.anchor, cfg.passing, cfg.n_text), world)
+    assert plan.shard_owners(world, "longest_first") == want.tolist()
+    if 8 % (2 * world) == 0:
+        assert plan.shard_owners(world, "zigzag") == orc.zigzag_owners(8, world).tolist()
+    assert plan.shard_owners(world if 8 % world == 0 else 1, "contiguous") == \
+        orc.contiguous_owners(8, world if 8 % world == 0 else 1).tolist()
     plan.close()

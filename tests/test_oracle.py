@@ -559,3 +559,36 @@ def test_sharded_attention_equals_single(policy, head_reduce):
     O, L = orc.sharded_attention(q, k, v, res["offsets"], cfg.anchor, res["sel"], scale, owner)
     np.testing.assert_allclose(O, res["O"], rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(L, res["lse"], rtol=1e-12, atol=1e-12)
+
+
+def test_host_costs_count_attended_pairs():
+    """Summed over the hosts, the per-host costs are the (query, key) pairs the
+    approximate attention evaluates: counted here row by row from the key sets."""
+    sizes, A, P, T = [40, 24, 56, 32], 6, 5, 9
+    N = sum(sizes)
+    off = orc.host_offsets(sizes)
+    sel = np.zeros((len(sizes) - 1, 1, P), dtype=np.int64)
+    for h in range(len(sizes) - 1):
+        lo = int(off[h]) + (A if h == 0 else 0)
+        sel[h, 0] = np.arange(lo, lo + P)
+    pairs = sum(len(orc.key_set(off, A, sel, 0, i, N)) for i in range(N + T))
+    cost = orc.host_costs(sizes, A, P, T)
+    assert int(cost.sum()) == pairs
+    assert (np.diff(orc.host_costs([32] * 6, A, P, 0)) > 0).all()   # later hosts carry more
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+def test_longest_first_within_graham_bound_of_optimum(world, seed):
+    """Longest-first list scheduling: every rank's load is at most the mean plus the
+    largest cost, and the largest load is within 4/3 - 1/(3W) of the optimum, found here
+    by trying every assignment (Graham's bound for this rule)."""
+    import itertools
+    rng = np.random.default_rng(seed)
+    cost = rng.integers(1, 50, size=7)
+    own = orc.longest_first_owners(cost, world)
+    load = np.bincount(own, weights=cost, minlength=world)
+    assert load.max() <= cost.sum() / world + cost.max()
+    best = min(np.bincount(np.array(a), weights=cost, minlength=world).max()
+               for a in itertools.product(range(world), repeat=len(cost)))
+    assert load.max() <= (4 / 3 - 1 / (3 * world)) * best + 1e-9

@@ -165,3 +165,19 @@ def test_sharded_orchestration_two_gloo_ranks(owner):
                 assert (o[h * B:(h + 1) * B] == r + 1).all()
                 assert (h * B, (h + 1) * B) in rows
         assert (o[64:] == 99).all()
+
+
+@pytest.mark.parametrize("W", [1, 2, 3, 8])
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_owners_by_cost_match_oracle(lib, W, seed):
+    """spava_shard_owners_by_cost (longest first) against the oracle's, integer for
+    integer, with many equal costs (ties go to the lower host, then the lower rank)."""
+    rng = np.random.default_rng(seed)
+    H = 16
+    cost = rng.integers(0, 6, size=H).astype(np.int64) * 1000
+    arr_c = (ctypes.c_int64 * H)(*[int(x) for x in cost])
+    out = (ctypes.c_int32 * H)()
+    assert lib.spava_shard_owners_by_cost(H, W, arr_c, out) == _lib.SPAVA_OK
+    assert list(out) == orc.longest_first_owners(cost, W).tolist()
+    arr_c[3] = -1
+    assert lib.spava_shard_owners_by_cost(H, W, arr_c, out) == _lib.SPAVA_ERR_INVALID_ARG
