@@ -48,6 +48,7 @@ CASES = {
     "prob_w2": (BASE, None, [0, 1, 1, 0], "max", "prob"),
     "one_host": (BASE.with_(n_hosts=1), None, [0], "max", "logit"),
     "no_anchor_no_passing_w2": (BASE.with_(anchor=0, passing=0), None, [0, 1, 1, 0], "max", "logit"),
+    "idle_rank_w3": (BASE, None, [0, 0, 2, 2], "max", "logit"),   # rank 1 runs no host
     # owners from the oracle's longest-first rule on these uneven blocks (3 ranks)
     "longest_first_w3_uneven": (BASE.with_(n_hosts=8, head_dim=64, anchor=16, passing=48),
                                 [96, 160, 128, 112, 144, 128, 100, 156], "longest_first:3", "max", "logit"),
