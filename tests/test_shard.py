@@ -181,3 +181,51 @@ def test_owners_by_cost_match_oracle(lib, W, seed):
     assert list(out) == orc.longest_first_owners(cost, W).tolist()
     arr_c[3] = -1
     assert lib.spava_shard_owners_by_cost(H, W, arr_c, out) == _lib.SPAVA_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------------ a rank that fails
+def _failing_rank_main(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from sequence_approximate_attention_b200.sharded import ShardedPrefill
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    log = []
+    plan = StandInPlan(4, 3, 64, 5, log)
+    sp = ShardedPrefill(plan, rank, world, [0, 1, 1, 0])
+    q, k, v = torch.zeros(69, 2, 4), torch.zeros(69, 1, 4), torch.zeros(69, 1, 4)
+    if rank == 1:
+        out[rank] = "left before the exchange"
+        os._exit(0)   # leaves between steps: none of its collectives is in flight
+    try:
+        sp.forward(q, k, v)
+        out[rank] = "finished"
+    except RuntimeError as e:
+        out[rank] = "error: " + type(e).__name__
+    os._exit(0)
+
+
+def test_surviving_rank_gets_an_error_not_a_hang():
+    """Failure on the host side: rank 1 leaves before the first exchange; rank 0's
+    all-gather ends with an error within the process group's short timeout instead of
+    waiting for ever."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as man:
+        out = man.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_failing_rank_main, args=(r, world, port, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+        alive = [p.is_alive() for p in procs]
+        for p in procs:
+            if p.is_alive():
+                p.kill()
+        res = dict(out)
+    assert not any(alive), "a rank hung"
+    assert res.get(1) == "left before the exchange"
+    assert res.get(0, "").startswith("error"), res
