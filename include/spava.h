@@ -367,6 +367,12 @@ spava_status spava_shard_query(const spava_plan* plan, spava_shard_layout* out);
  *                       Needs the gathered pass_k / pass_v and the anchor rows.
  *   SPAVA_SHARD_MERGE   text rows from all ranks' text slots (needs the gathered
  *                       text_o / text_lse): final O/lse of rows [N, N+T).
+ * One-pass form: SELECT, the passing exchange and the anchor broadcast (waited for),
+ * then SPAVA_SHARD_ATTEND in place of LOCAL + REMOTE -- own hosts' rows in one pass
+ * over [anchor | passing of hosts < h | own block, causal] (final O/lse, no row
+ * partials) and the text pieces into this rank's slots -- then the text exchange and
+ * MERGE.  It gives up overlapping the passing exchange with the local pass and saves
+ * the fp32 row partials and the second online softmax.
  * q, k, v, o [N+T][heads][d] bf16 and lse [hq][N+T] are full-size device buffers with
  * the layouts above.  Rows a rank does not own are not written and do not change the
  * result, but they must hold finite values (zeros will do): a 128-row tile can load
@@ -378,7 +384,8 @@ typedef enum {
   SPAVA_SHARD_SELECT = 0,
   SPAVA_SHARD_LOCAL = 1,
   SPAVA_SHARD_REMOTE = 2,
-  SPAVA_SHARD_MERGE = 3
+  SPAVA_SHARD_MERGE = 3,
+  SPAVA_SHARD_ATTEND = 4
 } spava_shard_stage_id;
 
 spava_status spava_shard_stage(const spava_plan* plan, int32_t stage, const void* q, const void* k,

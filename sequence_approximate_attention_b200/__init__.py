@@ -347,9 +347,9 @@ def shard_owners(n_hosts: int, world: int, policy: str = "zigzag"):
 def shard_stage(plan: Plan, stage: int, q: Optional[torch.Tensor], k: Optional[torch.Tensor],
                 v: Optional[torch.Tensor], o: Optional[torch.Tensor], lse: Optional[torch.Tensor],
                 workspace: torch.Tensor, stream=None) -> None:
-    """spava_shard_stage: one stage (SPAVA_SHARD_SELECT / LOCAL / REMOTE / MERGE) of the
-    sharded prefill on full-size q/k/v/o/lse buffers; see include/spava.h for which rows
-    each stage reads and writes."""
+    """spava_shard_stage: one stage (SPAVA_SHARD_SELECT / LOCAL / REMOTE / MERGE, or
+    ATTEND in place of LOCAL + REMOTE) of the sharded prefill on full-size q/k/v/o/lse
+    buffers; see include/spava.h for which rows each stage reads and writes."""
     dev = plan.device
     if stage != _lib.SPAVA_SHARD_MERGE:
         plan._check_qkv(q, k, v)

@@ -19,7 +19,7 @@ SPAVA_SCORES_GIVEN = 1
 SPAVA_SHARD_CONTIGUOUS = 0
 SPAVA_SHARD_ZIGZAG = 1
 SPAVA_SHARD_LONGEST_FIRST = 2
-SPAVA_SHARD_SELECT, SPAVA_SHARD_LOCAL, SPAVA_SHARD_REMOTE, SPAVA_SHARD_MERGE = 0, 1, 2, 3
+SPAVA_SHARD_SELECT, SPAVA_SHARD_LOCAL, SPAVA_SHARD_REMOTE, SPAVA_SHARD_MERGE, SPAVA_SHARD_ATTEND = 0, 1, 2, 3, 4
 
 
 class ShardLayout(ctypes.Structure):

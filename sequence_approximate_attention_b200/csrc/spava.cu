@@ -138,6 +138,8 @@ struct spava_plan {
   int n_items_shard_remote = 0;
   AttnItem* d_items_shard_probe = nullptr;
   int n_items_shard_probe = 0;
+  AttnItem* d_items_shard_pre = nullptr;  // one-pass form (SPAVA_SHARD_ATTEND)
+  int n_items_shard_pre = 0;
   // workspace layout
   size_t ws_err = 0, ws_scores = 0, ws_idx = 0, ws_kp = 0, ws_vp = 0, ws_opart = 0, ws_lpart = 0, ws_total = 0;
   size_t ws_row_o = 0, ws_row_lse = 0, ws_qkeys = 0, ws_total_two_stage = 0;  // two-stage flow only
@@ -244,11 +246,14 @@ void add_text_items(const spava_plan& p, std::vector<AttnItem>& v, std::vector<i
 // Work list of the prefill.  Host h's rows go in 256-row items per query head with
 // the KV list [anchor | passing of hosts < h | own block, causal]; text rows (the
 // query block) are split over the host blocks plus their own causal part, each
-// piece writing an fp32 partial with its lse.
-std::vector<AttnItem> build_prefill_items(const spava_plan& p) {
+// piece writing an fp32 partial with its lse.  With a host mask (sharded prefill)
+// only those hosts' rows and text pieces, into the given text slots.
+std::vector<AttnItem> build_prefill_items(const spava_plan& p, const HostMask* mine = nullptr,
+                                          const std::vector<int>* text_slot = nullptr) {
   std::vector<AttnItem> v;
   std::vector<int> group;
   for (int h = 0; h < p.H; ++h) {
+    if (!runs(mine, h)) continue;
     const int a = p.off[h], e = p.off[h + 1];
     for (int r0 = a; r0 < e; r0 += 256) {
       const int rows = std::min(256, e - r0);
@@ -263,7 +268,7 @@ std::vector<AttnItem> build_prefill_items(const spava_plan& p) {
       }
     }
   }
-  add_text_items(p, v, group);
+  add_text_items(p, v, group, text_slot);
   sort_host_major(v, group, p.hq / p.hkv);
   return v;
 }
@@ -1168,6 +1173,7 @@ spava_status spava_plan_set_shard(spava_plan* p, int32_t rank, int32_t world, co
   }
   const auto local = build_local_items(*p, &mine, &tslot);
   const auto remote = build_remote_items(*p, &mine);
+  const auto pre = build_prefill_items(*p, &mine, &tslot);
   const auto probe = build_probe_items(*p, H - 1, &mine);
   const auto score = passing ? build_score_items(*p, H - 1, &mine) : std::vector<int4>();
   TablePacker tab;
@@ -1177,6 +1183,7 @@ spava_status spava_plan_set_shard(spava_plan* p, int32_t rank, int32_t world, co
   const size_t o_local = tab.put(local.data(), local.size() * sizeof(AttnItem));
   const size_t o_remote = tab.put(remote.data(), remote.size() * sizeof(AttnItem));
   const size_t o_probe = tab.put(probe.data(), probe.size() * sizeof(AttnItem));
+  const size_t o_pre = tab.put(pre.data(), pre.size() * sizeof(AttnItem));
   if (p->dtab_shard) {
     SPAVA_CUDA(cudaDeviceSynchronize());
     SPAVA_CUDA(cudaFree(p->dtab_shard));
@@ -1205,6 +1212,8 @@ spava_status spava_plan_set_shard(spava_plan* p, int32_t rank, int32_t world, co
   p->n_items_shard_remote = static_cast<int>(remote.size());
   p->d_items_shard_probe = reinterpret_cast<AttnItem*>(base + o_probe);
   p->n_items_shard_probe = static_cast<int>(probe.size());
+  p->d_items_shard_pre = reinterpret_cast<AttnItem*>(base + o_pre);
+  p->n_items_shard_pre = static_cast<int>(pre.size());
   layout_workspace(p);
   return ok();
 }
@@ -1235,7 +1244,7 @@ spava_status spava_shard_stage(const spava_plan* p, int32_t stage, const void* q
   spava_status s;
   if ((s = check_plan_ws(p, ws)) != SPAVA_OK) return s;
   if (p->shard_world == 0) return fail(SPAVA_ERR_INVALID_ARG, "plan is not sharded (spava_plan_set_shard)");
-  if (stage < SPAVA_SHARD_SELECT || stage > SPAVA_SHARD_MERGE) return fail(SPAVA_ERR_INVALID_ARG, "unknown stage %d", stage);
+  if (stage < SPAVA_SHARD_SELECT || stage > SPAVA_SHARD_ATTEND) return fail(SPAVA_ERR_INVALID_ARG, "unknown stage %d", stage);
   const bool need_qkv = stage != SPAVA_SHARD_MERGE, need_o = stage != SPAVA_SHARD_SELECT;
   if (need_qkv && (!q || !k || !v)) return fail(SPAVA_ERR_INVALID_ARG, "NULL q, k or v");
   if (need_o && (!o || !lse)) return fail(SPAVA_ERR_INVALID_ARG, "NULL o or lse");
@@ -1250,6 +1259,36 @@ spava_status spava_shard_stage(const spava_plan* p, int32_t stage, const void* q
   ts.text_o = reinterpret_cast<float*>(w + p->ws_to);
   ts.text_lse = reinterpret_cast<float*>(w + p->ws_tl);
   const size_t pass_part = static_cast<size_t>(p->pass_slots) * p->P * score_rows(*p) * p->d * 2;
+  // this rank's unused text slots: O = 0, lse = -inf
+  auto fill_spare_text = [&]() -> spava_status {
+    const int spare = p->text_slots - p->text_slots_used;
+    if (p->T == 0 || spare <= 0) return SPAVA_OK;
+    const size_t slot0 = static_cast<size_t>(p->shard_rank) * p->text_slots + p->text_slots_used;
+    const size_t n_o = static_cast<size_t>(spare) * p->T * p->hq * p->d, n_l = static_cast<size_t>(spare) * p->hq * p->T;
+    uint32_t* fo = reinterpret_cast<uint32_t*>(ts.text_o) + slot0 * p->T * p->hq * p->d;
+    uint32_t* fl = reinterpret_cast<uint32_t*>(ts.text_lse) + slot0 * p->hq * p->T;
+    const int grid = std::max(1, std::min(p->num_sms * 4, static_cast<int>((n_o + 255) / 256)));
+    mark(p, kLabFill, st);
+    spava::fill_u32_kernel<<<grid, 256, 0, st>>>(fo, n_o, 0u);
+    spava::fill_u32_kernel<<<grid, 256, 0, st>>>(fl, n_l, 0xFF800000u);
+    SPAVA_CUDA(cudaGetLastError());
+    g_last_launches += 2;
+    return SPAVA_OK;
+  };
+  // every host's passing rows from the gathered exchange buffers into k_pass / v_pass
+  auto unpack = [&]() -> spava_status {
+    if (!scores_needed(*p)) return SPAVA_OK;
+    const int rows = score_rows(*p), cpr = p->d * 2 / 16;
+    const size_t total = static_cast<size_t>(rows) * (p->H - 1) * p->P * cpr;
+    const int grid = static_cast<int>(std::min<size_t>((total + 255) / 256, static_cast<size_t>(p->num_sms) * 8));
+    mark(p, kLabUnpack, st);
+    spava::unpack_passing_kernel<<<grid, 256, 0, st>>>(
+        reinterpret_cast<const uint4*>(w + p->ws_xk), reinterpret_cast<const uint4*>(w + p->ws_xv), p->d_xrow0,
+        reinterpret_cast<uint4*>(w + p->ws_kp), reinterpret_cast<uint4*>(w + p->ws_vp), rows, p->H - 1, p->P, cpr);
+    SPAVA_CUDA(cudaGetLastError());
+    ++g_last_launches;
+    return SPAVA_OK;
+  };
   switch (stage) {
     case SPAVA_SHARD_SELECT: {
       if (!scores_needed(*p) || p->n_shard_hosts == 0) break;
@@ -1265,19 +1304,7 @@ spava_status spava_shard_stage(const spava_plan* p, int32_t stage, const void* q
       break;
     }
     case SPAVA_SHARD_LOCAL: {
-      const int spare = p->text_slots - p->text_slots_used;
-      if (p->T > 0 && spare > 0) {  // this rank's unused text slots: O = 0, lse = -inf
-        const size_t slot0 = static_cast<size_t>(p->shard_rank) * p->text_slots + p->text_slots_used;
-        const size_t n_o = static_cast<size_t>(spare) * p->T * p->hq * p->d, n_l = static_cast<size_t>(spare) * p->hq * p->T;
-        uint32_t* fo = reinterpret_cast<uint32_t*>(ts.text_o) + slot0 * p->T * p->hq * p->d;
-        uint32_t* fl = reinterpret_cast<uint32_t*>(ts.text_lse) + slot0 * p->hq * p->T;
-        const int grid = std::max(1, std::min(p->num_sms * 4, static_cast<int>((n_o + 255) / 256)));
-        mark(p, kLabFill, st);
-        spava::fill_u32_kernel<<<grid, 256, 0, st>>>(fo, n_o, 0u);
-        spava::fill_u32_kernel<<<grid, 256, 0, st>>>(fl, n_l, 0xFF800000u);
-        SPAVA_CUDA(cudaGetLastError());
-        g_last_launches += 2;
-      }
+      if ((s = fill_spare_text()) != SPAVA_OK) return s;
       s = p->d == 128 ? launch_attn<128>(p, p->d_items_shard_local, p->n_items_shard_local, q, k, v, nullptr, nullptr,
                                          o, lse, ws, st, ts)
                       : launch_attn<64>(p, p->d_items_shard_local, p->n_items_shard_local, q, k, v, nullptr, nullptr,
@@ -1289,21 +1316,23 @@ spava_status spava_shard_stage(const spava_plan* p, int32_t stage, const void* q
       if (p->n_items_shard_remote == 0) break;
       void* kp = w + p->ws_kp;
       void* vp = w + p->ws_vp;
-      if (scores_needed(*p)) {
-        const int rows = score_rows(*p), cpr = p->d * 2 / 16;
-        const size_t total = static_cast<size_t>(rows) * (p->H - 1) * p->P * cpr;
-        const int grid = static_cast<int>(std::min<size_t>((total + 255) / 256, static_cast<size_t>(p->num_sms) * 8));
-        mark(p, kLabUnpack, st);
-        spava::unpack_passing_kernel<<<grid, 256, 0, st>>>(
-            reinterpret_cast<const uint4*>(w + p->ws_xk), reinterpret_cast<const uint4*>(w + p->ws_xv), p->d_xrow0,
-            static_cast<uint4*>(kp), static_cast<uint4*>(vp), rows, p->H - 1, p->P, cpr);
-        SPAVA_CUDA(cudaGetLastError());
-        ++g_last_launches;
-      }
+      if ((s = unpack()) != SPAVA_OK) return s;
       s = p->d == 128 ? launch_attn<128>(p, p->d_items_shard_remote, p->n_items_shard_remote, q, k, v, kp, vp, o, lse,
                                          ws, st, ts)
                       : launch_attn<64>(p, p->d_items_shard_remote, p->n_items_shard_remote, q, k, v, kp, vp, o, lse,
                                         ws, st, ts);
+      if (s != SPAVA_OK) return s;
+      break;
+    }
+    case SPAVA_SHARD_ATTEND: {
+      if ((s = fill_spare_text()) != SPAVA_OK) return s;
+      void* kp = w + p->ws_kp;
+      void* vp = w + p->ws_vp;
+      if (p->n_items_shard_remote > 0 && (s = unpack()) != SPAVA_OK) return s;
+      s = p->d == 128 ? launch_attn<128>(p, p->d_items_shard_pre, p->n_items_shard_pre, q, k, v, kp, vp, o, lse, ws,
+                                         st, ts)
+                      : launch_attn<64>(p, p->d_items_shard_pre, p->n_items_shard_pre, q, k, v, kp, vp, o, lse, ws,
+                                        st, ts);
       if (s != SPAVA_OK) return s;
       break;
     }

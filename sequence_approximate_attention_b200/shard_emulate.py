@@ -3,7 +3,8 @@
     python -m sequence_approximate_attention_b200.shard_emulate --config 128k \\
         --worlds 2,4,8 --policies zigzag,contiguous,longest_first
 
-For each (world W, ownership policy) it builds the W ranks' plans on this GPU, runs
+For each (world W, ownership policy, form: LOCAL + REMOTE or the one-pass ATTEND)
+it builds the W ranks' plans on this GPU, runs
 their stages in the order a W-GPU job would (every rank's SELECT, the exchange, every
 LOCAL, the text exchange, every REMOTE, every MERGE), moving the exchanged bytes with
 device copies between the stages, and times every kernel of each rank with the
@@ -13,7 +14,8 @@ stages of different ranks alternate on the GPU, so each stage starts with anothe
 rank's data in L2 (no L2 reuse between a rank's stages is assumed).  The collectives
 themselves are not timed (one GPU); the bytes each rank contributes are reported.
 
-One JSON line per (W, policy): per-rank compute, its max and mean, the balance
+One JSON line per (W, policy, form): per-rank compute (its select, attention and merge
+parts), its max and mean, the balance
 (max / mean), the one-GPU spava_attn_prefill time on the same inputs, and the
 compute-only speed-up that the slowest rank allows.
 """
@@ -28,11 +30,15 @@ import torch
 
 from . import Plan, _lib, attn_prefill, shard_stage
 
-STAGES = (_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_LOCAL, _lib.SPAVA_SHARD_REMOTE, _lib.SPAVA_SHARD_MERGE)
-STAGE_NAMES = ("select", "local", "remote", "merge")
-# the stage each kernel of the timing hook belongs to
-KERNEL_STAGE = {"probe_lse": 0, "score": 0, "select_gather": 0, "score_keys": 1, "attention_local": 1,
-                "unpack_passing": 2, "attention_remote": 2, "lse_merge": 3}
+FLOWS = {
+    "two_stage": (_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_LOCAL, _lib.SPAVA_SHARD_REMOTE, _lib.SPAVA_SHARD_MERGE),
+    "one_pass": (_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_ATTEND, _lib.SPAVA_SHARD_MERGE),
+}
+# the part of a layer each kernel of the timing hook belongs to
+KERNEL_PART = {"probe_lse": "select", "score": "select", "select_gather": "select", "score_keys": "attention",
+               "attention_local": "attention", "unpack_passing": "attention", "attention_remote": "attention",
+               "attention": "attention", "lse_merge": "merge"}
+PARTS = ("select", "attention", "merge")
 
 
 def _workloads():
@@ -48,7 +54,7 @@ def _plan(cfg, sizes, dev):
                 cfg.head_dim, device=dev)
 
 
-def emulate(cfg, sizes, q, k, v, world, policy, steps, warmup):
+def emulate(cfg, sizes, q, k, v, world, policy, steps, warmup, flow="two_stage"):
     dev = q.device
     probe = _plan(cfg, sizes, dev)
     owner = probe.shard_owners(world, policy)
@@ -72,13 +78,13 @@ def emulate(cfg, sizes, q, k, v, world, policy, steps, warmup):
                     S["ws"][off + r * per: off + (r + 1) * per].copy_(part)
 
     def layer():
-        for sid in STAGES:
+        for sid in FLOWS[flow]:
             for R in ranks:
                 shard_stage(R["plan"], sid, q, k, v, o, lse, R["ws"])
             if sid == _lib.SPAVA_SHARD_SELECT:
                 exchange(L0.pass_k_offset, L0.pass_bytes_per_rank)
                 exchange(L0.pass_v_offset, L0.pass_bytes_per_rank)
-            elif sid == _lib.SPAVA_SHARD_LOCAL:
+            elif sid in (_lib.SPAVA_SHARD_LOCAL, _lib.SPAVA_SHARD_ATTEND):
                 exchange(L0.text_o_offset, L0.text_o_bytes_per_rank)
                 exchange(L0.text_lse_offset, L0.text_lse_bytes_per_rank)
 
@@ -90,10 +96,10 @@ def emulate(cfg, sizes, q, k, v, world, policy, steps, warmup):
     for _ in range(steps):
         layer()
     torch.cuda.synchronize(dev)
-    per_stage = np.zeros((world, len(STAGES)))   # [rank][stage] ms per layer
+    per_stage = np.zeros((world, len(PARTS)))   # [rank][part] ms per layer
     for r, R in enumerate(ranks):
         for name, ms in R["plan"].profile_read():
-            per_stage[r, KERNEL_STAGE[name]] += ms / steps
+            per_stage[r, PARTS.index(KERNEL_PART[name])] += ms / steps
         R["plan"].profile_end()
         R["plan"].close()
     per_rank = per_stage.sum(axis=1)
@@ -101,7 +107,7 @@ def emulate(cfg, sizes, q, k, v, world, policy, steps, warmup):
     return {
         "owner": owner,
         "rank_ms": [round(float(x), 4) for x in per_rank],
-        "stage_ms": {n: [round(float(x), 4) for x in per_stage[:, i]] for i, n in enumerate(STAGE_NAMES)},
+        "part_ms": {n: [round(float(x), 4) for x in per_stage[:, i]] for i, n in enumerate(PARTS)},
         "max_ms": float(per_rank.max()), "mean_ms": float(per_rank.mean()),
         "balance": float(per_rank.max() / per_rank.mean()),
         "exchange_bytes_per_rank": {"passing_kv": 2 * int(L0.pass_bytes_per_rank),
@@ -133,6 +139,7 @@ def main(argv=None):
     ap.add_argument("--config", default="128k", choices=sorted(CONFIGS))
     ap.add_argument("--worlds", default="2,4,8")
     ap.add_argument("--policies", default="zigzag,contiguous,longest_first")
+    ap.add_argument("--flows", default="two_stage,one_pass")
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     args = ap.parse_args(argv)
@@ -142,20 +149,20 @@ def main(argv=None):
     dev = torch.device("cuda", torch.cuda.current_device())
     q, k, v = (torch.from_numpy(g[x].view(np.int16)).view(torch.bfloat16).to(dev) for x in ("q", "k", "v"))
     base = one_gpu_ms(cfg, sizes, q, k, v, args.steps, args.warmup)
-    for world in (int(x) for x in args.worlds.split(",")):
-        for policy in args.policies.split(","):
-            try:
-                res = emulate(cfg, sizes, q, k, v, world, policy, args.steps, args.warmup)
-            except (ValueError, _lib.SpavaError) as e:
-                print(json.dumps({"config": cfg.name, "world": world, "policy": policy, "skipped": str(e)}))
-                continue
-            res.update({"metric": "sharded prefill: per-rank compute, ranks emulated on one GPU",
-                        "unit": "ms", "config": cfg.name, "world": world, "policy": policy,
-                        "one_gpu_prefill_ms": round(base, 4),
-                        "compute_speedup_vs_one_gpu": round(base / res["max_ms"], 3),
-                        "ideal_speedup": world})
-            print(json.dumps(res), flush=True)
-
+    combos = [(int(w), p, f) for w in args.worlds.split(",") for p in args.policies.split(",")
+              for f in args.flows.split(",")]
+    for world, policy, flow in combos:
+        try:
+            res = emulate(cfg, sizes, q, k, v, world, policy, args.steps, args.warmup, flow)
+        except (ValueError, _lib.SpavaError) as e:
+            print(json.dumps({"config": cfg.name, "world": world, "policy": policy, "skipped": str(e)}))
+            continue
+        res.update({"metric": "sharded prefill: per-rank compute, ranks emulated on one GPU",
+                    "unit": "ms", "config": cfg.name, "world": world, "policy": policy, "flow": flow,
+                    "one_gpu_prefill_ms": round(base, 4),
+                    "compute_speedup_vs_one_gpu": round(base / res["max_ms"], 3),
+                    "ideal_speedup": world})
+        print(json.dumps(res), flush=True)
 
 if __name__ == "__main__":
     main()

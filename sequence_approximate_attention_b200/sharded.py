@@ -17,6 +17,11 @@ while attention computes.  Per rank and layer:
             merged with the local partials
     MERGE   (waits for the text partials) text rows from all ranks' slots
 
+With ``overlap=False`` (the one-pass form) the rank waits for the passing exchange
+after SELECT and runs ATTEND, one pass per own host over [anchor | passing | own
+block], instead of LOCAL + REMOTE: on NVLink the exchange is short next to the
+attention, and one pass saves the fp32 row partials and the second online softmax.
+
 Every rank issues the same collectives in the same order.  The exchange buffers
 live in the plan's sharded workspace, rank-major, so every collective is an
 in-place all-gather of one contiguous run per rank.  With NCCL they run on a
@@ -38,10 +43,11 @@ __all__ = ["ShardedPrefill"]
 class ShardedPrefill:
     """One rank's side of the sharded prefill of a plan (see the module docstring)."""
 
-    def __init__(self, plan, rank: int, world: int, owner: Sequence[int], group=None):
+    def __init__(self, plan, rank: int, world: int, owner: Sequence[int], group=None, overlap: bool = True):
         if len(owner) != plan.n_hosts:
             raise ValueError("owner needs one rank per host")
         self.plan, self.rank, self.world, self.group = plan, int(rank), int(world), group
+        self.overlap = bool(overlap)
         self.owner = [int(x) for x in owner]
         plan.set_shard(self.rank, self.world, self.owner)
         L = plan.shard_layout()
@@ -115,11 +121,17 @@ class ShardedPrefill:
             k.record_stream(self.comm)
             v.record_stream(self.comm)
         pass_done = self._on_comm(mark(), self._exchange_passing, k, v)
-        plan.shard_stage(_lib.SPAVA_SHARD_LOCAL, q, k, v, o, lse, self.ws)
-        text_done = self._on_comm(mark(), self._exchange_text)
-        if pass_done is not None:
-            cur.wait_event(pass_done)
-        plan.shard_stage(_lib.SPAVA_SHARD_REMOTE, q, k, v, o, lse, self.ws)
+        if self.overlap:
+            plan.shard_stage(_lib.SPAVA_SHARD_LOCAL, q, k, v, o, lse, self.ws)
+            text_done = self._on_comm(mark(), self._exchange_text)
+            if pass_done is not None:
+                cur.wait_event(pass_done)
+            plan.shard_stage(_lib.SPAVA_SHARD_REMOTE, q, k, v, o, lse, self.ws)
+        else:
+            if pass_done is not None:
+                cur.wait_event(pass_done)
+            plan.shard_stage(_lib.SPAVA_SHARD_ATTEND, q, k, v, o, lse, self.ws)
+            text_done = self._on_comm(mark(), self._exchange_text)
         if text_done is not None:
             cur.wait_event(text_done)
         plan.shard_stage(_lib.SPAVA_SHARD_MERGE, None, None, None, o, lse, self.ws)

@@ -250,7 +250,8 @@ def test_fullsize_score_variants_qwen64k(reduce, kind):
     torch.cuda.empty_cache()
 
 
-def test_fullsize_sharded_emulated(fullsize_run):
+@pytest.mark.parametrize("flow", ["two_stage", "one_pass"])
+def test_fullsize_sharded_emulated(fullsize_run, flow):
     """The sharded prefill at full size, its W ranks run one after another on this GPU
     (128k: W = 8, ZigZag; stress: W = 4, ZigZag, uneven blocks), the exchange moved by
     device copies between the stages: every host's selection equals the one-GPU
@@ -281,13 +282,15 @@ def test_fullsize_sharded_emulated(fullsize_run):
                     ws2[off + rk * per: off + (rk + 1) * per].copy_(ws[off + rk * per: off + (rk + 1) * per])
 
     from sequence_approximate_attention_b200 import _lib
-    for sid in (_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_LOCAL, _lib.SPAVA_SHARD_REMOTE, _lib.SPAVA_SHARD_MERGE):
+    stages = ((_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_LOCAL, _lib.SPAVA_SHARD_REMOTE, _lib.SPAVA_SHARD_MERGE)
+              if flow == "two_stage" else (_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_ATTEND, _lib.SPAVA_SHARD_MERGE))
+    for sid in stages:
         for p, _, ws in ranks:
             sab.shard_stage(p, sid, dev["q"], dev["k"], dev["v"], o, lse, ws)
         if sid == _lib.SPAVA_SHARD_SELECT:
             exchange(L0.pass_k_offset, L0.pass_bytes_per_rank)
             exchange(L0.pass_v_offset, L0.pass_bytes_per_rank)
-        elif sid == _lib.SPAVA_SHARD_LOCAL:
+        elif sid in (_lib.SPAVA_SHARD_LOCAL, _lib.SPAVA_SHARD_ATTEND):
             exchange(L0.text_o_offset, L0.text_o_bytes_per_rank)
             exchange(L0.text_lse_offset, L0.text_lse_bytes_per_rank)
     for p, _, ws in ranks:

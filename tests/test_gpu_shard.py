@@ -1,5 +1,6 @@
 """GPU parity of the sharded prefill's stages (spava_plan_set_shard / spava_shard_stage),
-with the ranks emulated one after another on one GPU.
+in both forms (LOCAL + REMOTE, or the one-pass ATTEND), with the ranks emulated one
+after another on one GPU.
 
 Every emulated rank has its own plan, workspace and full-size q/k/v/o/lse buffers in
 which only its own host rows and the text rows hold the inputs; every other row holds
@@ -68,7 +69,7 @@ def _garbage_like(t, rng_seed):
     return (torch.randn(t.shape, generator=g) * 40.0).to(torch.bfloat16).to(t.device)
 
 
-def _run_emulated(name):
+def _run_emulated(name, flow="two_stage"):
     cfg, sizes, owner, mode, kind = CASES[name]
     cfg = cfg.with_(uneven=None)
     g, f64, dev = inputs(cfg)
@@ -118,10 +119,15 @@ def _run_emulated(name):
     for R in ranks:
         R["k"][:A] = src["k"][:A]
         R["v"][:A] = src["v"][:A]
-    stage(_lib.SPAVA_SHARD_LOCAL)
-    allgather("text_o_offset", "text_o_bytes_per_rank")
-    allgather("text_lse_offset", "text_lse_bytes_per_rank")
-    stage(_lib.SPAVA_SHARD_REMOTE)
+    if flow == "two_stage":
+        stage(_lib.SPAVA_SHARD_LOCAL)
+        allgather("text_o_offset", "text_o_bytes_per_rank")
+        allgather("text_lse_offset", "text_lse_bytes_per_rank")
+        stage(_lib.SPAVA_SHARD_REMOTE)
+    else:
+        stage(_lib.SPAVA_SHARD_ATTEND)
+        allgather("text_o_offset", "text_o_bytes_per_rank")
+        allgather("text_lse_offset", "text_lse_bytes_per_rank")
     stage(_lib.SPAVA_SHARD_MERGE)
     for R in ranks:
         sab.check_device_error(R["plan"], R["ws"])
@@ -129,9 +135,10 @@ def _run_emulated(name):
     return cfg, f64, dev, sizes, off, owner, ranks
 
 
+@pytest.mark.parametrize("flow", ["two_stage", "one_pass"])
 @pytest.mark.parametrize("name", list(CASES))
-def test_sharded_stages_match_oracle(name):
-    cfg, f64, dev, sizes, off, owner, ranks = _run_emulated(name)
+def test_sharded_stages_match_oracle(name, flow):
+    cfg, f64, dev, sizes, off, owner, ranks = _run_emulated(name, flow)
     H, N, NT = cfg.n_hosts, cfg.n_visual, cfg.n_total
     plan0 = ranks[0]["plan"]
     rows = plan0.score_rows

@@ -107,13 +107,16 @@ class StandInPlan:
         elif stage == _lib.SPAVA_SHARD_LOCAL:
             to[r] = 30 + r
             tl[r] = 40 + r
-        elif stage == _lib.SPAVA_SHARD_REMOTE:
+        elif stage in (_lib.SPAVA_SHARD_REMOTE, _lib.SPAVA_SHARD_ATTEND):
             for rr in range(self.world):
                 assert (pk[rr] == 10 + rr).all() and (pv[rr] == 20 + rr).all(), "passing exchange incomplete"
             assert (k[:self.anchor] == 7).all() and (v[:self.anchor] == 8).all(), "anchor rows missing"
             for h in range(self.n_hosts):
                 if self.owner[h] == r:
                     o[self.offsets[h]:self.offsets[h + 1]] = r + 1
+            if stage == _lib.SPAVA_SHARD_ATTEND:   # the one-pass form also fills the text slots
+                to[r] = 30 + r
+                tl[r] = 40 + r
         elif stage == _lib.SPAVA_SHARD_MERGE:
             for rr in range(self.world):
                 assert (to[rr] == 30 + rr).all() and (tl[rr] == 40 + rr).all(), "text exchange incomplete"
@@ -126,7 +129,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, owner, out):
+def _rank_main(rank, world, port, owner, overlap, out):
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
     from sequence_approximate_attention_b200.sharded import ShardedPrefill
@@ -135,7 +138,7 @@ def _rank_main(rank, world, port, owner, out):
     log = []
     H, A, N, T = len(owner), 3, 64, 5
     plan = StandInPlan(H, A, N, T, log)
-    sp = ShardedPrefill(plan, rank, world, owner)
+    sp = ShardedPrefill(plan, rank, world, owner, overlap=overlap)
     q = torch.zeros(N + T, 2, 4)
     k = torch.zeros(N + T, 1, 4)
     v = torch.zeros(N + T, 1, 4)
@@ -147,18 +150,20 @@ def _rank_main(rank, world, port, owner, out):
     dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("overlap", [True, False])
 @pytest.mark.parametrize("owner", [[0, 1, 1, 0], [1, 0, 0, 1], [0, 0, 1, 1]])
-def test_sharded_orchestration_two_gloo_ranks(owner):
+def test_sharded_orchestration_two_gloo_ranks(owner, overlap):
     world = 2
     with mp.get_context("spawn").Manager() as man:
         out = man.dict()
-        mp.spawn(_rank_main, args=(world, _free_port(), owner, out), nprocs=world, join=True)
+        mp.spawn(_rank_main, args=(world, _free_port(), owner, overlap, out), nprocs=world, join=True)
         res = dict(out)
     B = 64 // len(owner)
+    stages = ([_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_LOCAL, _lib.SPAVA_SHARD_REMOTE, _lib.SPAVA_SHARD_MERGE]
+              if overlap else [_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_ATTEND, _lib.SPAVA_SHARD_MERGE])
     for r in range(world):
         log, o, rows = res[r]
-        assert log == [_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_LOCAL, _lib.SPAVA_SHARD_REMOTE,
-                       _lib.SPAVA_SHARD_MERGE]
+        assert log == stages
         o = np.array(o)
         for h, own in enumerate(owner):
             if own == r:
