@@ -417,7 +417,8 @@ spava_status spava_profile_end(spava_plan* plan);
 /* Name of a kernel label: 0 score, 1 select, 2 gather, 3 attention (prefill),
  * 4 lse merge, 5 attention (dense causal), 6 select + gather (fused, prefill),
  * 7 score-key fill/convert (two-stage), 8 attention stage 1, 9 attention stage 2,
- * 10 probe-row lse (probability scores), 11 passing unpack (sharded prefill). */
+ * 10 probe-row lse (probability scores), 11 passing unpack (sharded prefill),
+ * 12 spare text-slot fill (sharded prefill). */
 const char* spava_kernel_name(int32_t label);
 
 /* Static text of a status code. */

@@ -161,7 +161,7 @@ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 enum KernelLabel {
   kLabScore = 0, kLabSelect = 1, kLabGather = 2, kLabAttn = 3, kLabMerge = 4, kLabDense = 5, kLabSelectGather = 6,
-  kLabFill = 7, kLabAttnLocal = 8, kLabAttnRemote = 9, kLabProbeLse = 10, kLabUnpack = 11
+  kLabFill = 7, kLabAttnLocal = 8, kLabAttnRemote = 9, kLabProbeLse = 10, kLabUnpack = 11, kLabTextFill = 12
 };
 
 void mark(const spava_plan* p, int label, cudaStream_t st) {
@@ -687,14 +687,16 @@ spava_status upload_table(const std::vector<uint8_t>& host, void** out) {
   return SPAVA_OK;
 }
 
-// Packs arrays into one host image for upload_table, each 256-byte aligned.
+// Packs arrays into one host image for upload_table, each 256-byte aligned.  An
+// empty array still takes a slot, so no two arrays share an address (the kernel
+// timing labels tell work lists apart by address).
 struct TablePacker {
   std::vector<uint8_t> host;
   size_t put(const void* src, size_t bytes) {
     const size_t at = host.size();
     const uint8_t* b = static_cast<const uint8_t*>(src);
     if (bytes) host.insert(host.end(), b, b + bytes);
-    host.resize(align_up(host.size(), 256), 0);
+    host.resize(align_up(at + std::max<size_t>(bytes, 1), 256), 0);
     return at;
   }
 };
@@ -805,25 +807,17 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   p->n_score_pre = static_cast<int>(sc_pre.size());
   p->n_score_all = static_cast<int>(sc_all.size());
   // One device table, each array 256-byte aligned.
-  std::vector<uint8_t> host;
-  auto put = [&host](const void* src, size_t bytes) {
-    const size_t at = host.size();
-    host.resize(align_up(at + bytes, 256), 0);
-    if (bytes) std::memcpy(host.data() + at, src, bytes);
-    return at;
-  };
-  const size_t o_off = put(off.data(), off.size() * 4);
-  const size_t o_pre = put(pre.data(), pre.size() * sizeof(AttnItem));
-  const size_t o_dense = put(dense.data(), dense.size() * sizeof(AttnItem));
-  const size_t o_spre = put(sc_pre.data(), sc_pre.size() * sizeof(int4));
-  const size_t o_sall = put(sc_all.data(), sc_all.size() * sizeof(int4));
-  const size_t o_local = put(local.data(), local.size() * sizeof(AttnItem));
-  const size_t o_remote = put(remote.data(), remote.size() * sizeof(AttnItem));
-  const size_t o_probe = put(probe.data(), probe.size() * sizeof(AttnItem));
-  e = cudaMalloc(&p->dtab, host.size());
-  if (e != cudaSuccess) return bail(fail(SPAVA_ERR_CUDA, "cudaMalloc(plan table): %s", cudaGetErrorString(e)));
-  e = cudaMemcpy(p->dtab, host.data(), host.size(), cudaMemcpyHostToDevice);
-  if (e != cudaSuccess) return bail(fail(SPAVA_ERR_CUDA, "cudaMemcpy(plan table): %s", cudaGetErrorString(e)));
+  TablePacker tab;
+  const size_t o_off = tab.put(off.data(), off.size() * 4);
+  const size_t o_pre = tab.put(pre.data(), pre.size() * sizeof(AttnItem));
+  const size_t o_dense = tab.put(dense.data(), dense.size() * sizeof(AttnItem));
+  const size_t o_spre = tab.put(sc_pre.data(), sc_pre.size() * sizeof(int4));
+  const size_t o_sall = tab.put(sc_all.data(), sc_all.size() * sizeof(int4));
+  const size_t o_local = tab.put(local.data(), local.size() * sizeof(AttnItem));
+  const size_t o_remote = tab.put(remote.data(), remote.size() * sizeof(AttnItem));
+  const size_t o_probe = tab.put(probe.data(), probe.size() * sizeof(AttnItem));
+  spava_status ust = upload_table(tab.host, &p->dtab);
+  if (ust != SPAVA_OK) return bail(ust);
   uint8_t* base = static_cast<uint8_t*>(p->dtab);
   p->d_off = reinterpret_cast<int*>(base + o_off);
   p->d_items_pre = reinterpret_cast<AttnItem*>(base + o_pre);
@@ -1268,7 +1262,7 @@ spava_status spava_shard_stage(const spava_plan* p, int32_t stage, const void* q
     uint32_t* fo = reinterpret_cast<uint32_t*>(ts.text_o) + slot0 * p->T * p->hq * p->d;
     uint32_t* fl = reinterpret_cast<uint32_t*>(ts.text_lse) + slot0 * p->hq * p->T;
     const int grid = std::max(1, std::min(p->num_sms * 4, static_cast<int>((n_o + 255) / 256)));
-    mark(p, kLabFill, st);
+    mark(p, kLabTextFill, st);
     spava::fill_u32_kernel<<<grid, 256, 0, st>>>(fo, n_o, 0u);
     spava::fill_u32_kernel<<<grid, 256, 0, st>>>(fl, n_l, 0xFF800000u);
     SPAVA_CUDA(cudaGetLastError());
@@ -1399,6 +1393,7 @@ const char* spava_kernel_name(int32_t label) {
     case kLabAttnRemote: return "attention_remote";
     case kLabProbeLse: return "probe_lse";
     case kLabUnpack: return "unpack_passing";
+    case kLabTextFill: return "text_slot_fill";
   }
   return "unknown";
 }

@@ -37,7 +37,7 @@ FLOWS = {
 # the part of a layer each kernel of the timing hook belongs to
 KERNEL_PART = {"probe_lse": "select", "score": "select", "select_gather": "select", "score_keys": "attention",
                "attention_local": "attention", "unpack_passing": "attention", "attention_remote": "attention",
-               "attention": "attention", "lse_merge": "merge"}
+               "attention": "attention", "text_slot_fill": "attention", "lse_merge": "merge"}
 PARTS = ("select", "attention", "merge")
 
 

@@ -222,3 +222,23 @@ def test_plan_owners_match_oracle(world):
     assert plan.shard_owners(world if 8 % world == 0 else 1, "contiguous") == \
         orc.contiguous_owners(8, world if 8 % world == 0 else 1).tolist()
     plan.close()
+
+
+def test_stage_kernel_labels_for_a_rank_without_scored_hosts():
+    """Rank 0 runs only the last host (nothing to score): SELECT launches nothing and
+    the timing hook names ATTEND's kernels as the unpack and the attention (its empty
+    work lists must not share an address with the one it runs)."""
+    cfg = BASE
+    plan = make_plan(sab, cfg, [256] * 4)
+    plan.set_shard(0, 2, [1, 1, 1, 0])
+    g, _, dev = inputs(cfg)
+    ws = torch.zeros(plan.shard_workspace_bytes, dtype=torch.uint8, device="cuda")
+    o = torch.zeros_like(dev["q"])
+    lse = torch.zeros((cfg.hq, cfg.n_total), device="cuda")
+    plan.profile_begin(64)
+    for sid in (_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_ATTEND, _lib.SPAVA_SHARD_MERGE):
+        sab.shard_stage(plan, sid, dev["q"], dev["k"], dev["v"], o, lse, ws)
+    names = [n for n, _ in plan.profile_read()]
+    plan.profile_end()
+    assert names == ["text_slot_fill", "unpack_passing", "attention", "lse_merge"], names
+    plan.close()
