@@ -8,9 +8,9 @@ the later hosts and its partial query results to be merged, and these transfers 
 while attention computes.  Per rank and layer:
 
     compute stream                         comm stream
+                                           broadcast anchor rows k, v [0, A)
     SELECT  score/select own hosts,
             passing rows -> own part  ---> all-gather passing K, V
-                                           broadcast anchor rows k, v [0, A)
     LOCAL   own blocks (causal),
             text pieces -> own slots  ---> all-gather text partials (O, lse)
     REMOTE  (waits for the passing and anchor) own hosts over [anchor | passing],
@@ -72,13 +72,17 @@ class ShardedPrefill:
         if whole.numel():
             dist.all_gather_into_tensor(whole, mine, group=self.group)
 
-    def _exchange_passing(self, k: torch.Tensor, v: torch.Tensor) -> None:
-        self._gather(self.pass_k, self.pass_k_mine)
-        self._gather(self.pass_v, self.pass_v_mine)
+    def _broadcast_anchor(self, k: torch.Tensor, v: torch.Tensor) -> None:
+        # rows [0, A) belong to host 0: read by its owner's stages only, written here
+        # on every other rank, where no stage before REMOTE / ATTEND reads them
         A = self.plan.anchor
         if A > 0 and self.plan.n_hosts > 1:
             dist.broadcast(k[:A], src=self.anchor_src, group=self.group)
             dist.broadcast(v[:A], src=self.anchor_src, group=self.group)
+
+    def _exchange_passing(self) -> None:
+        self._gather(self.pass_k, self.pass_k_mine)
+        self._gather(self.pass_v, self.pass_v_mine)
 
     def _exchange_text(self) -> None:
         self._gather(self.text_o, self.text_o_mine)
@@ -116,11 +120,12 @@ class ShardedPrefill:
             e.record(cur)
             return e
 
-        plan.shard_stage(_lib.SPAVA_SHARD_SELECT, q, k, v, None, None, self.ws)
         if self.cuda:
             k.record_stream(self.comm)
             v.record_stream(self.comm)
-        pass_done = self._on_comm(mark(), self._exchange_passing, k, v)
+        self._on_comm(mark(), self._broadcast_anchor, k, v)
+        plan.shard_stage(_lib.SPAVA_SHARD_SELECT, q, k, v, None, None, self.ws)
+        pass_done = self._on_comm(mark(), self._exchange_passing)
         if self.overlap:
             plan.shard_stage(_lib.SPAVA_SHARD_LOCAL, q, k, v, o, lse, self.ws)
             text_done = self._on_comm(mark(), self._exchange_text)
