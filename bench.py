@@ -300,6 +300,78 @@ def workload_config(cfg):
             "l2": "inputs larger than L2 (no flush)", "parallelism": "replicas"}
 
 
+# ---------------------------------------------------------------- sharded prefill
+def run_sharded(args, cfg, rank, world, local):
+    """--sharded POLICY: the layer's hosts spread over the N ranks (ShardedPrefill, NCCL
+    exchange), total work fixed (strong scaling).  Every rank generates the same
+    seeded workload and uses its own host rows and the text rows; the anchor rows
+    arrive by broadcast.  value = the layer's N+T tokens per step over the max-over-ranks
+    time."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import sequence_approximate_attention_b200 as sab
+    from sequence_approximate_attention_b200.sharded import ShardedPrefill
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world == 1 and "MASTER_ADDR" not in os.environ:
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK="0", WORLD_SIZE="1")
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    g = generate(cfg)
+    sizes = [int(x) for x in g["host_sizes"]]
+    NT = cfg.n_visual + cfg.n_text
+    d_in = {x: torch.from_numpy(g[x].view(np.int16)).view(torch.bfloat16).to(dev) for x in ("q", "k", "v")}
+    plan = sab.Plan(cfg.n_visual, cfg.n_text, cfg.n_hosts, sizes, cfg.anchor, cfg.passing, cfg.probe_r,
+                    cfg.hq, cfg.hkv, cfg.head_dim, device=dev)
+    owner = plan.shard_owners(world, args.sharded)
+    sp = ShardedPrefill(plan, rank, world, owner, overlap=args.sharded_form == "overlap")
+    o = torch.empty_like(d_in["q"])
+    lse = torch.empty((cfg.hq, NT), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(args.warmup, 3)):
+        sp.forward(d_in["q"], d_in["k"], d_in["v"], o, lse)
+    sab.check_device_error(plan, sp.ws)
+    clocks = ClockSampler(str(torch.cuda.get_device_properties(dev).uuid))
+    clocks.start()
+    time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = sp.launches
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        sp.forward(d_in["q"], d_in["k"], d_in["v"], o, lse)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clk = clocks.stop()
+    sab.check_device_error(plan, sp.ws)
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), dev)
+    if rank == 0:
+        conf = workload_config(cfg)
+        conf.update({"parallelism": f"sharded-{args.sharded}-{args.sharded_form}", "owner": owner,
+                     "l2": "inputs larger than L2 (no flush)"})
+        line = {"metric": METRIC, "value": NT * args.steps / (ms_total / 1e3), "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_total / args.steps,
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic", "impl": "b200", "config": conf, "roofline": None, "cpu_baseline": None,
+                "e2e": None, "gpu_launches": sp.launches - launches0, "clocks": clk,
+                "note": "one layer's hosts spread over the ranks; inputs resident on every rank; the exchange "
+                        "(NCCL all-gathers and broadcast) inside the timed region"}
+        print(json.dumps(line), flush=True)
+    del sp
+    dist.barrier()
+    dist.destroy_process_group()
+    plan.close()
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -321,6 +393,10 @@ def main():
     ap.add_argument("--cpu-baseline", type=int, default=1)
     ap.add_argument("--cpu-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=256)
+    ap.add_argument("--sharded", default=None, choices=["zigzag", "contiguous", "longest_first"],
+                    help="instead of replicas: one layer's hosts spread over the N ranks with this ownership "
+                         "(strong scaling)")
+    ap.add_argument("--sharded-form", default="overlap", choices=["overlap", "one_pass"])
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
 
@@ -331,6 +407,9 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, cfg)
+        return
+    if args.sharded:
+        run_sharded(args, cfg, rank, world, local)
         return
 
     import torch

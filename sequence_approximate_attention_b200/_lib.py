@@ -112,6 +112,11 @@ def load(build_if_missing: bool = True):
     return lib
 
 
+def launches_of_last_call() -> int:
+    """spava_last_launch_count, or 0 where the library is not loaded (stand-in plans)."""
+    return int(_LIB.spava_last_launch_count()) if _LIB is not None else 0
+
+
 def check(status: int, where: str) -> None:
     if status != SPAVA_OK:
         detail = load().spava_last_error().decode(errors="replace")

@@ -66,6 +66,7 @@ class ShardedPrefill:
         self.anchor_src = self.owner[0]
         self.cuda = plan.device.type == "cuda"
         self.comm = torch.cuda.Stream(device=plan.device) if self.cuda else None
+        self.launches = 0  # library kernel launches enqueued by forward() so far
 
     # -- collectives (same sequence on every rank)
     def _gather(self, whole: torch.Tensor, mine: torch.Tensor) -> None:
@@ -112,6 +113,11 @@ class ShardedPrefill:
         if lse is None:
             lse = torch.empty((plan.hq, plan.n_total), dtype=torch.float32, device=plan.device)
         cur = torch.cuda.current_stream(plan.device) if self.cuda else None
+        stage_fn = plan.shard_stage
+
+        def stage(*a):
+            stage_fn(*a)
+            self.launches += _lib.launches_of_last_call()
 
         def mark():
             if not self.cuda:
@@ -124,22 +130,22 @@ class ShardedPrefill:
             k.record_stream(self.comm)
             v.record_stream(self.comm)
         self._on_comm(mark(), self._broadcast_anchor, k, v)
-        plan.shard_stage(_lib.SPAVA_SHARD_SELECT, q, k, v, None, None, self.ws)
+        stage(_lib.SPAVA_SHARD_SELECT, q, k, v, None, None, self.ws)
         pass_done = self._on_comm(mark(), self._exchange_passing)
         if self.overlap:
-            plan.shard_stage(_lib.SPAVA_SHARD_LOCAL, q, k, v, o, lse, self.ws)
+            stage(_lib.SPAVA_SHARD_LOCAL, q, k, v, o, lse, self.ws)
             text_done = self._on_comm(mark(), self._exchange_text)
             if pass_done is not None:
                 cur.wait_event(pass_done)
-            plan.shard_stage(_lib.SPAVA_SHARD_REMOTE, q, k, v, o, lse, self.ws)
+            stage(_lib.SPAVA_SHARD_REMOTE, q, k, v, o, lse, self.ws)
         else:
             if pass_done is not None:
                 cur.wait_event(pass_done)
-            plan.shard_stage(_lib.SPAVA_SHARD_ATTEND, q, k, v, o, lse, self.ws)
+            stage(_lib.SPAVA_SHARD_ATTEND, q, k, v, o, lse, self.ws)
             text_done = self._on_comm(mark(), self._exchange_text)
         if text_done is not None:
             cur.wait_event(text_done)
-        plan.shard_stage(_lib.SPAVA_SHARD_MERGE, None, None, None, o, lse, self.ws)
+        stage(_lib.SPAVA_SHARD_MERGE, None, None, None, o, lse, self.ws)
         return o, lse
 
     def owned_rows(self):
