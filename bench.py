@@ -300,6 +300,34 @@ def workload_config(cfg):
             "l2": "inputs larger than L2 (no flush)", "parallelism": "replicas"}
 
 
+def init_nccl(dev, world):
+    """NCCL process group bound to `dev`.  The communicator comes up eagerly here, with
+    file descriptor 1 pointed at stderr meanwhile: the library prints a version banner
+    on rank 0 from C, and stdout must carry only the one JSON line."""
+    import contextlib
+    import datetime
+
+    import torch.distributed as dist
+
+    @contextlib.contextmanager
+    def stdout_to_stderr():
+        sys.stdout.flush()
+        saved = os.dup(1)
+        os.dup2(2, 1)
+        try:
+            yield
+        finally:
+            sys.stdout.flush()
+            import ctypes
+            ctypes.CDLL(None).fflush(None)   # C stdio buffers written while fd 1 was stderr
+            os.dup2(saved, 1)
+            os.close(saved)
+
+    with stdout_to_stderr():
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        dist.barrier()
+
+
 # ---------------------------------------------------------------- sharded prefill
 def run_sharded(args, cfg, rank, world, local):
     """--sharded POLICY: the layer's hosts spread over the N ranks (ShardedPrefill, NCCL
@@ -307,8 +335,6 @@ def run_sharded(args, cfg, rank, world, local):
     seeded workload and uses its own host rows and the text rows; the anchor rows
     arrive by broadcast.  value = the layer's N+T tokens per step over the max-over-ranks
     time."""
-    import datetime
-
     import torch
     import torch.distributed as dist
 
@@ -323,7 +349,7 @@ def run_sharded(args, cfg, rank, world, local):
             sk.bind(("127.0.0.1", 0))
             port = sk.getsockname()[1]
         os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK="0", WORLD_SIZE="1")
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    init_nccl(dev, world)
     g = generate(cfg)
     sizes = [int(x) for x in g["host_sizes"]]
     NT = cfg.n_visual + cfg.n_text
@@ -414,15 +440,13 @@ def main():
 
     import torch
     import torch.distributed as dist
-    import datetime
 
     import sequence_approximate_attention_b200 as sab
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        init_nccl(dev, world)
 
     def barrier():
         if world > 1:
