@@ -515,7 +515,7 @@ def main():
             gbs = sgb[name] / (avg[name] / 1e3) / 1e9
             hbm[name] = {"ms": avg[name], "bytes": sgb[name], "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]}
     if "score" in hbm:
-        # the score kernel sits at its ridge point: report the tensor side too
+        # the score kernel also does 64 GFLOP of MMAs at 128k: report its tensor side too
         sf = score_flops(cfg, sizes)
         hbm["score"]["flops"] = sf
         hbm["score"]["TFLOP/s"] = sf / (avg["score"] / 1e3) / 1e12
