@@ -57,6 +57,7 @@ def test_shard_owners_refuse_bad_sizes(lib, H, W, policy):
 def test_set_shard_refuses_null_plan(lib):
     arr = (ctypes.c_int32 * 2)(0, 0)
     assert lib.spava_plan_set_shard(None, 0, 1, arr) == _lib.SPAVA_ERR_INVALID_ARG
+    assert lib.spava_plan_shard_owners(None, 2, _lib.SPAVA_SHARD_LONGEST_FIRST, arr) == _lib.SPAVA_ERR_INVALID_ARG
     assert lib.spava_shard_query(None, None) == _lib.SPAVA_ERR_INVALID_ARG
     assert lib.spava_shard_stage(None, 0, None, None, None, None, None, None, None) == _lib.SPAVA_ERR_INVALID_ARG
 
