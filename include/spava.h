@@ -214,9 +214,12 @@ spava_status spava_attn_prefill(const spava_plan* plan, const void* q, const voi
  * allocating library routine); the inputs and outputs are the caller's, with the
  * layouts of spava_attn_prefill.  The plan must have been created beforehand
  * (spava_plan_create allocates its table once, at set-up).
- *   First call on a device: it looks up the array's device address on the current
- *   device (cudaGetSymbolAddress) and caches it; make that first call before any
- *   stream capture.
+ *   Address: every call looks up the array's device address on the current device
+ *   (cudaGetSymbolAddress, a host-side lookup that enqueues nothing) and caches
+ *   nothing, so a context torn down and re-created in the same process
+ *   (cudaDeviceReset) gets the array's new address.  With lazy module loading the
+ *   first lookup on a device loads the library's kernels there: make that first call
+ *   before any stream capture.
  *   Sizes: returns SPAVA_ERR_UNSUPPORTED, before enqueueing anything, when
  *   spava_workspace_bytes(plan) exceeds SPAVA_NOALLOC_SCRATCH_BYTES.
  *   Sharing: every call on a device uses the same array, which keeps the previous

@@ -954,24 +954,17 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[SPAVA_NOALLOC_S
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mutex;
-void* g_noalloc_addr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on device `dev` (which must be current): in
-// host code the symbol is only a host-side stand-in, so the address is looked up
-// once per device and cached.
-spava_status noalloc_scratch_address(int dev, void** out) {
-  if (dev < 0 || dev >= kMaxDevices) return fail(SPAVA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_addr[dev]) {
-    void* addr = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
-    if (e != cudaSuccess || !addr)
-      return fail(SPAVA_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
-    g_noalloc_addr[dev] = addr;
-  }
-  *out = g_noalloc_addr[dev];
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// symbol is only a host-side stand-in, so the address is looked up on every call:
+// the lookup enqueues nothing, and a cached address would go stale if the device's
+// context were torn down and re-created (cudaDeviceReset reloads the module, and the
+// array may then sit elsewhere).
+spava_status noalloc_scratch_address(void** out) {
+  void* addr = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
+  if (e != cudaSuccess || !addr)
+    return fail(SPAVA_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
+  *out = addr;
   return SPAVA_OK;
 }
 
@@ -991,7 +984,7 @@ spava_status spava_attn_prefill_noalloc(const spava_plan* p, const void* q, cons
   SPAVA_CUDA(cudaGetDevice(&dev));
   if (dev != p->device) return fail(SPAVA_ERR_INVALID_ARG, "current device %d differs from the plan's device %d", dev, p->device);
   void* ws = nullptr;
-  spava_status s = noalloc_scratch_address(dev, &ws);
+  spava_status s = noalloc_scratch_address(&ws);
   if (s != SPAVA_OK) return s;
   return spava_attn_prefill(p, q, k, v, o, lse, nullptr, nullptr, ws, stream);
 }
