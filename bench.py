@@ -222,37 +222,52 @@ class LazyF64:
         return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
 
 
-def oracle_sample(cfg, g, seed, rows=512):
-    """One bounded oracle run: probe scoring + top-P selection of every host, then
-    the blockwise attention of one `rows`-row slice of a random host (all heads).
-    Returns (seconds for the whole workload, extrapolated by attended key pairs;
-    description; seconds actually spent)."""
+def oracle_sample(cfg, g, seed, rows=64):
+    """One bounded oracle run on a fixed stratified sample of the layer: probe scoring
+    and top-P selection of every host in full, then the attention of one `rows`-row
+    slice of every host block and of the text rows (all heads), each slice at a
+    seeded position inside its stratum.  Each stratum is extrapolated by its own
+    attended key pairs (remote-heavy late hosts and the dense text rows cost
+    differently per row).  Returns (seconds for the whole layer; description;
+    seconds actually spent; fraction of the layer's attended pairs computed)."""
     from oracle import spava_oracle as orc
     q, k, v = LazyF64(g["q"]), LazyF64(g["k"]), LazyF64(g["v"])
     sizes = [int(x) for x in g["host_sizes"]]
     off = orc.host_offsets(sizes)
     scale = 1.0 / math.sqrt(cfg.head_dim)
+    N, T, A, P = cfg.n_visual, cfg.n_text, cfg.anchor, cfg.passing
     t0 = time.perf_counter()
     sel = None
     if cfg.n_hosts > 1:
         scores = orc.probe_scores(q, k, off, cfg.probe_r, scale)
-        sel = orc.select_passing(scores, off, cfg.anchor, cfg.passing)
+        sel = orc.select_passing(scores, off, A, P)
     t_sel = time.perf_counter() - t0
     rng = np.random.default_rng(seed)
-    h = int(rng.integers(0, cfg.n_hosts))
-    a, e = int(off[h]), int(off[h + 1])
-    r0 = a + int(rng.integers(0, max(1, e - a - rows + 1)))
-    r1 = min(e, r0 + rows)
-    remote = (cfg.anchor + h * cfg.passing) if h >= 1 else 0
-    pairs_sample = sum(remote + (i - a + 1) for i in range(r0, r1))
-    t1 = time.perf_counter()
-    orc.approx_attention(q, k, v, off, cfg.anchor, sel, scale, row_range=(r0, r1))
-    t_att = time.perf_counter() - t1
-    total = t_sel + t_att * attended_pairs(cfg, sizes) / pairs_sample
-    desc = (f"fp64 numpy oracle: probe scoring + top-P selection of all hosts ({t_sel:.2f} s), then the "
-            f"blockwise attention of rows {r0}..{r1 - 1} (host {h}, all {cfg.hq} heads, {t_att:.2f} s), "
-            f"extrapolated to the whole layer by attended key pairs")
-    return total, desc, t_sel + t_att
+    # strata: (first row, end row, keys before the stratum's causal part per row)
+    strata = [(int(off[h]), int(off[h + 1]), (A + h * P) if h >= 1 else 0) for h in range(cfg.n_hosts)]
+    if T > 0:
+        strata.append((N, N + T, N))
+    t_att, t_total, pairs_done = 0.0, t_sel, 0
+    for a, e, remote in strata:
+        n = min(rows, e - a)
+        r0 = a + int(rng.integers(0, e - a - n + 1))
+        r1 = r0 + n
+        # pairs of a row i: the remote keys plus its causal part; text rows see [0, i]
+        pairs_of = (lambda i: i + 1) if a == N else (lambda i: remote + (i - a + 1))
+        sample = sum(pairs_of(i) for i in range(r0, r1))
+        stratum = sum(pairs_of(i) for i in range(a, e))
+        t1 = time.perf_counter()
+        orc.approx_attention(q, k, v, off, A, sel, scale, row_range=(r0, r1), compact=True)
+        dt = time.perf_counter() - t1
+        t_att += dt
+        t_total += dt * stratum / sample
+        pairs_done += sample
+    frac = pairs_done / attended_pairs(cfg, sizes)
+    desc = (f"fp64 numpy oracle: probe scoring + top-P selection of all {cfg.n_hosts} hosts in full "
+            f"({t_sel:.2f} s), then one {rows}-row slice (all {cfg.hq} heads, seeded position) of every host "
+            f"block{' and of the text rows' if T > 0 else ''} ({t_att:.2f} s, {100 * frac:.2f} % of the layer's "
+            f"attended pairs), each slice extrapolated by its own stratum's attended pairs")
+    return t_total, desc, t_sel + t_att, frac
 
 
 def blas_threads():
@@ -270,12 +285,11 @@ def run_reference(args, cfg):
     for w in range(args.warmup):
         oracle_sample(cfg, g, 100 + w, rows=args.ref_rows)
     times = []
-    descs = []
     wall = 0.0
+    desc, frac = "", 0.0
     for s in range(args.steps):
-        t, desc, w = oracle_sample(cfg, g, 1000 + s, rows=args.ref_rows)
+        t, desc, w, frac = oracle_sample(cfg, g, 1000 + s, rows=args.ref_rows)
         times.append(t)
-        descs.append(desc)
         wall += w
     t_step = statistics.median(times)
     value = NT / t_step
@@ -284,9 +298,12 @@ def run_reference(args, cfg):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "ms_per_step_kind": "extrapolated: each step computes a stratified sample of the layer and scales it by "
+                            "attended pairs; not a wall time per step",
+        "sampled_wall_s_per_step": wall / max(1, args.steps), "sampled_fraction_of_layer": frac,
         "config": workload_config(cfg),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": descs[-1] + f"; median of {args.steps} samples, {wall:.1f} s of CPU work"},
+                         "sample": desc + f"; median of {args.steps} samples (seeds 1000..), {wall:.1f} s of CPU work"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -398,6 +415,139 @@ def run_sharded(args, cfg, rank, world, local):
     plan.close()
 
 
+# ---------------------------------------------------------------- sharded prefill, ranks emulated
+# the part of a layer each kernel of the timing hook belongs to
+KERNEL_PART = {"probe_lse": "select", "score": "select", "select_gather": "select", "score_keys": "attention",
+               "attention_local": "attention", "unpack_passing": "attention", "attention_remote": "attention",
+               "attention": "attention", "text_slot_fill": "attention", "lse_merge": "merge"}
+PARTS = ("select", "attention", "merge")
+
+
+def shard_emulate(cfg, sizes, q, k, v, world, policy, steps, warmup, flow):
+    """Per-rank compute of the sharded prefill with the W ranks emulated on one GPU:
+    every rank's plan runs its stages in the order a W-GPU job would (every SELECT,
+    the exchange, every LOCAL (or ATTEND), the text exchange, every REMOTE, every
+    MERGE), the exchanged bytes moved by device copies between the stages, every
+    kernel of each rank timed by the library's timing hook (CUDA events on the
+    launching stream).  A rank's compute is the sum of its kernel times: what its own
+    GPU would spend.  The collectives are not timed (one GPU)."""
+    import torch
+
+    import sequence_approximate_attention_b200 as sab
+    from sequence_approximate_attention_b200 import _lib
+    flows = {"two_stage": (_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_LOCAL, _lib.SPAVA_SHARD_REMOTE,
+                           _lib.SPAVA_SHARD_MERGE),
+             "one_pass": (_lib.SPAVA_SHARD_SELECT, _lib.SPAVA_SHARD_ATTEND, _lib.SPAVA_SHARD_MERGE)}
+    dev = q.device
+
+    def new_plan():
+        return sab.Plan(cfg.n_visual, cfg.n_text, cfg.n_hosts, sizes, cfg.anchor, cfg.passing, cfg.probe_r,
+                        cfg.hq, cfg.hkv, cfg.head_dim, device=dev)
+
+    probe = new_plan()
+    owner = probe.shard_owners(world, policy)
+    probe.close()
+    ranks = []
+    for r in range(world):
+        p = new_plan()
+        p.set_shard(r, world, owner)
+        L = p.shard_layout()
+        ranks.append({"plan": p, "L": L, "ws": torch.zeros(int(L.workspace_bytes), dtype=torch.uint8, device=dev)})
+    o = torch.zeros_like(q)
+    lse = torch.zeros((cfg.hq, cfg.n_visual + cfg.n_text), dtype=torch.float32, device=dev)
+    L0 = ranks[0]["L"]
+
+    def exchange(off, per):
+        off, per = int(off), int(per)
+        for r, R in enumerate(ranks):
+            part = R["ws"][off + r * per: off + (r + 1) * per]
+            for S in ranks:
+                if S is not R:
+                    S["ws"][off + r * per: off + (r + 1) * per].copy_(part)
+
+    def layer():
+        for sid in flows[flow]:
+            for R in ranks:
+                sab.shard_stage(R["plan"], sid, q, k, v, o, lse, R["ws"])
+            if sid == _lib.SPAVA_SHARD_SELECT:
+                exchange(L0.pass_k_offset, L0.pass_bytes_per_rank)
+                exchange(L0.pass_v_offset, L0.pass_bytes_per_rank)
+            elif sid in (_lib.SPAVA_SHARD_LOCAL, _lib.SPAVA_SHARD_ATTEND):
+                exchange(L0.text_o_offset, L0.text_o_bytes_per_rank)
+                exchange(L0.text_lse_offset, L0.text_lse_bytes_per_rank)
+
+    for _ in range(warmup):
+        layer()
+    torch.cuda.synchronize(dev)
+    for R in ranks:
+        R["plan"].profile_begin(steps * 16 + 16)
+    for _ in range(steps):
+        layer()
+    torch.cuda.synchronize(dev)
+    per_stage = np.zeros((world, len(PARTS)))   # [rank][part] ms per layer
+    for r, R in enumerate(ranks):
+        for name, ms in R["plan"].profile_read():
+            per_stage[r, PARTS.index(KERNEL_PART[name])] += ms / steps
+        R["plan"].profile_end()
+        R["plan"].close()
+    per_rank = per_stage.sum(axis=1)
+    anchor_bytes = 2 * cfg.anchor * cfg.hkv * cfg.head_dim * 2
+    return {
+        "owner": owner,
+        "rank_ms": [round(float(x), 4) for x in per_rank],
+        "part_ms": {n: [round(float(x), 4) for x in per_stage[:, i]] for i, n in enumerate(PARTS)},
+        "max_ms": float(per_rank.max()), "mean_ms": float(per_rank.mean()),
+        "balance": float(per_rank.max() / per_rank.mean()),
+        "exchange_bytes_per_rank": {"passing_kv": 2 * int(L0.pass_bytes_per_rank),
+                                    "text_partials": int(L0.text_o_bytes_per_rank + L0.text_lse_bytes_per_rank),
+                                    "anchor_broadcast": anchor_bytes},
+    }
+
+
+def run_shard_emulate(args, cfg):
+    """--shard-emulate: one JSON line per (world W, ownership policy, form): per-rank
+    compute (select, attention and merge parts), its max and mean, the balance
+    (max / mean), the one-GPU spava_attn_prefill time on the same inputs and the
+    compute-only speed-up the slowest rank allows.  Not the bench contract's line."""
+    import torch
+
+    import sequence_approximate_attention_b200 as sab
+    g = generate(cfg)
+    sizes = [int(x) for x in g["host_sizes"]]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v = (torch.from_numpy(g[x].view(np.int16)).view(torch.bfloat16).to(dev) for x in ("q", "k", "v"))
+    p = sab.Plan(cfg.n_visual, cfg.n_text, cfg.n_hosts, sizes, cfg.anchor, cfg.passing, cfg.probe_r,
+                 cfg.hq, cfg.hkv, cfg.head_dim, device=dev)
+    ws = p.new_workspace()
+    o = torch.empty_like(q)
+    lse = torch.empty((cfg.hq, cfg.n_visual + cfg.n_text), dtype=torch.float32, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        sab.attn_prefill(p, q, k, v, o=o, lse=lse, workspace=ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        sab.attn_prefill(p, q, k, v, o=o, lse=lse, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    base = e0.elapsed_time(e1) / args.steps
+    p.close()
+    del ws
+    combos = [(int(w), pol, f) for w in args.worlds.split(",") for pol in args.policies.split(",")
+              for f in args.flows.split(",")]
+    for world, policy, flow in combos:
+        try:
+            res = shard_emulate(cfg, sizes, q, k, v, world, policy, args.steps, max(args.warmup, 3), flow)
+        except (ValueError, sab.SpavaError) as e:
+            print(json.dumps({"config": cfg.name, "world": world, "policy": policy, "skipped": str(e)}))
+            continue
+        res.update({"metric": "sharded prefill: per-rank compute, ranks emulated on one GPU",
+                    "unit": "ms", "config": cfg.name, "world": world, "policy": policy, "flow": flow,
+                    "one_gpu_prefill_ms": round(base, 4),
+                    "compute_speedup_vs_one_gpu": round(base / res["max_ms"], 3),
+                    "ideal_speedup": world})
+        print(json.dumps(res), flush=True)
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -417,12 +567,20 @@ def main():
                          "approximate vs dense")
     ap.add_argument("--dense", type=int, default=1, help="also time the dense causal kernel (0/1)")
     ap.add_argument("--cpu-baseline", type=int, default=1)
-    ap.add_argument("--cpu-rows", type=int, default=1024)
-    ap.add_argument("--ref-rows", type=int, default=256)
+    # rows per stratum (host block, text rows) of the oracle's sample; the same for both
+    # arms so their figures are comparable
+    ap.add_argument("--cpu-rows", type=int, default=64)
+    ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--sharded", default=None, choices=["zigzag", "contiguous", "longest_first"],
                     help="instead of replicas: one layer's hosts spread over the N ranks with this ownership "
                          "(strong scaling)")
     ap.add_argument("--sharded-form", default="overlap", choices=["overlap", "one_pass"])
+    ap.add_argument("--shard-emulate", action="store_true",
+                    help="instead of the bench line: the sharded prefill's per-rank compute with the ranks "
+                         "emulated on this one GPU, one JSON line per (world, policy, form)")
+    ap.add_argument("--worlds", default="2,4,8")
+    ap.add_argument("--policies", default="zigzag,contiguous,longest_first")
+    ap.add_argument("--flows", default="two_stage,one_pass")
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
 
@@ -436,6 +594,10 @@ def main():
         return
     if args.sharded:
         run_sharded(args, cfg, rank, world, local)
+        return
+    if args.shard_emulate:
+        if rank == 0:
+            run_shard_emulate(args, cfg)
         return
 
     import torch
@@ -632,9 +794,10 @@ def main():
 
     cpu = None
     if args.cpu_baseline and rank == 0 and world == 1:
-        t_full, desc, work = oracle_sample(cfg, g, 7, rows=args.cpu_rows)
+        t_full, desc, work, frac = oracle_sample(cfg, g, 7, rows=args.cpu_rows)
         cpu = {"value": NT / t_full, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": desc + f"; {work:.1f} s of CPU work", "host_cpus": os.cpu_count()}
+               "sample": desc + f"; seed 7, {work:.1f} s of CPU work", "host_cpus": os.cpu_count(),
+               "sampled_fraction_of_layer": frac}
 
     if rank == 0:
         line = {

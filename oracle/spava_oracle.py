@@ -200,13 +200,15 @@ def _masked_softmax_attend(logits: np.ndarray, visible: np.ndarray, vals: np.nda
 
 def approx_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, off: np.ndarray,
                      anchor: int, sel: Optional[np.ndarray], scale: float,
-                     row_chunk: int = 512, row_range=None):
+                     row_chunk: int = 512, row_range=None, compact: bool = False):
     """Approximate attention of every row (host blocks + trailing text rows).
 
     Host h >= 1 attends to [anchor | passing of hosts < h | own block, causal];
     host 0 and text rows attend densely and causally.  Returns O float64
     [tokens, hq, d] and lse float64 [hq, tokens] (natural log).  With
-    ``row_range=(r0, r1)`` only rows r0..r1-1 are computed (the rest stay NaN).
+    ``row_range=(r0, r1)`` only rows r0..r1-1 are computed (the rest stay NaN);
+    with ``compact`` as well, only those rows are stored: O [r1-r0, hq, d] and lse
+    [hq, r1-r0] (a storage choice, the arithmetic is the same).
     """
     NT, hq, d = q.shape
     hkv = k.shape[1]
@@ -214,8 +216,11 @@ def approx_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, off: np.ndarra
     H = len(off) - 1
     N = int(off[-1])
     lo_row, hi_row = (0, NT) if row_range is None else (int(row_range[0]), int(row_range[1]))
-    O = np.full((NT, hq, d), np.nan, dtype=np.float64)
-    lse = np.full((hq, NT), np.nan, dtype=np.float64)
+    compact = compact and row_range is not None
+    base = lo_row if compact else 0
+    n_out = hi_row - lo_row if compact else NT
+    O = np.full((n_out, hq, d), np.nan, dtype=np.float64)
+    lse = np.full((hq, n_out), np.nan, dtype=np.float64)
     for h in range(H):
         a, e = int(off[h]), int(off[h + 1])
         if e <= lo_row or a >= hi_row:
@@ -235,7 +240,7 @@ def approx_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, off: np.ndarra
                 visible[:, remote.size:] = np.arange(a, r1)[None, :] <= np.arange(r0, r1)[:, None]
                 kk, vv = k[keys, g, :], v[keys, g, :]
                 logits = np.matmul(q[r0:r1, c, :], kk.T) * scale
-                O[r0:r1, c], lse[c, r0:r1] = _masked_softmax_attend(logits, visible, vv)
+                O[r0 - base:r1 - base, c], lse[c, r0 - base:r1 - base] = _masked_softmax_attend(logits, visible, vv)
     for r0 in range(max(N, lo_row), min(NT, hi_row), row_chunk):
         r1 = min(NT, hi_row, r0 + row_chunk)
         keys = np.arange(0, r1)
@@ -244,7 +249,7 @@ def approx_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, off: np.ndarra
             kk, vv = k[:r1, g, :], v[:r1, g, :]
             for c in range(g * G, (g + 1) * G):
                 logits = np.matmul(q[r0:r1, c, :], kk.T) * scale
-                O[r0:r1, c], lse[c, r0:r1] = _masked_softmax_attend(logits, visible, vv)
+                O[r0 - base:r1 - base, c], lse[c, r0 - base:r1 - base] = _masked_softmax_attend(logits, visible, vv)
     return O, lse
 
 

@@ -257,6 +257,11 @@ def test_row_range_matches_full():
         np.testing.assert_allclose(O[r0:r1], full["O"][r0:r1], rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(L[:, r0:r1], full["lse"][:, r0:r1], rtol=1e-12, atol=1e-12)
         assert np.isnan(O[r1:]).all() and np.isnan(O[:r0]).all()
+        Oc, Lc = orc.approx_attention(q, k, v, full["offsets"], cfg.anchor, full["sel"], scale,
+                                      row_chunk=64, row_range=(r0, r1), compact=True)
+        assert Oc.shape == (r1 - r0,) + O.shape[1:] and Lc.shape == (L.shape[0], r1 - r0)
+        np.testing.assert_array_equal(Oc, O[r0:r1])
+        np.testing.assert_array_equal(Lc, L[:, r0:r1])
 
 
 # ---------------------------------------------------------------- brute force: scores, select
