@@ -3,10 +3,13 @@ configuration bench.py times (one plan, one workspace, one spava_attn_prefill).
 
 Every score of hosts 0..H-2 is checked against the fp64 oracle; the selection is
 checked bit-exactly against the oracle's selection on the GPU's own fp32 scores and
-for near-tie-only differences against the fp64 selection; O and lse are checked on
-sampled (row, head) outputs -- block starts, tile boundaries, probe rows, block
-ends, text rows and random rows -- against the oracle re-run with the GPU's
-indices.  The 256k workload also runs the dense causal kernel on the same inputs.
+for near-tie-only differences against the fp64 selection; O and lse are checked
+element by element, every head, on whole 128-row tiles of the kernel -- the first, a
+middle and the last tile of every host block -- and on every text row, against the
+oracle re-run with the GPU's indices (the oracle runs in a spawn-started process
+pool, tests/oracle_pool.py); further sampled (row, head) outputs cover block starts,
+tile boundaries, probe rows and random rows.  The 256k workload also runs the dense
+causal kernel on the same inputs, checked on four whole tiles.
 """
 
 import math
@@ -18,6 +21,7 @@ import torch
 from oracle import spava_oracle as orc
 from workloads import CONFIGS, generate
 
+from . import oracle_pool
 from .helpers import LSE_TOL, O_TOL, check_selection_vs_fp64, to_device_bf16
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
@@ -72,6 +76,36 @@ def _sample_rows(cfg, off, rng, n_random=48):
     rows = sorted(rows)
     heads = [int((i * 7 + 3) % cfg.hq) for i in range(len(rows))]
     return rows, heads
+
+
+def _whole_tiles(cfg, off):
+    """Row ranges of whole 128-row tiles of the attention kernel (tiles start at each
+    block's first row): the first, a middle and the last tile of every host block,
+    and all text rows."""
+    ranges = []
+    for h in range(cfg.n_hosts):
+        a, e = int(off[h]), int(off[h + 1])
+        B = e - a
+        for t in sorted({0, 128 * ((B // 128) // 2), 128 * ((B - 1) // 128)}):
+            ranges.append((a + t, min(e, a + t + 128)))
+    if cfg.n_text:
+        ranges.append((cfg.n_visual, cfg.n_visual + cfg.n_text))
+    return ranges
+
+
+def _compare_ranges(o_dev, lse_dev, ranges, refs, what):
+    """Every head of every row of the ranges against the oracle; returns the number of
+    (row, head) outputs compared."""
+    n, worst_o, worst_l = 0, 0.0, 0.0
+    for (r0, r1), (O_ref, L_ref) in zip(ranges, refs):
+        o = o_dev[r0:r1].float().cpu().numpy()
+        lse = lse_dev[:, r0:r1].cpu().numpy()
+        assert np.isfinite(o).all() and np.isfinite(lse).all(), (what, r0, r1)
+        worst_o = max(worst_o, float(np.abs(o - O_ref).max()))
+        worst_l = max(worst_l, float(np.abs(lse - L_ref).max()))
+        n += O_ref.shape[0] * O_ref.shape[1]
+    assert worst_o <= O_TOL and worst_l <= LSE_TOL, (what, n, worst_o, worst_l)
+    return n
 
 
 @pytest.fixture(scope="module", params=["qwen64k", "128k", "stress", "256k"])
@@ -137,6 +171,25 @@ def test_fullsize_sampled_outputs(fullsize_run):
     assert torch.isfinite(r["o"].float()).all().item() and torch.isfinite(r["lse"]).all().item()
 
 
+# (row, head) outputs compared element by element per workload: (tiles + text rows) x heads
+WHOLE_TILE_OUTPUTS = {"qwen64k": (24 * 128 + 128) * 28, "128k": (48 * 128 + 256) * 32,
+                      "stress": None, "256k": (96 * 128 + 256) * 32}
+
+
+def test_fullsize_whole_tiles(fullsize_run):
+    r = fullsize_run
+    cfg = r["cfg"]
+    off = orc.host_offsets(r["sizes"])
+    ranges = _whole_tiles(cfg, off)
+    refs = oracle_pool.attention_rows_ranges(r["g"], off, cfg.anchor, r["idx"], 1.0 / math.sqrt(cfg.head_dim),
+                                             ranges)
+    n = _compare_ranges(r["o"], r["lse"], ranges, refs, cfg.name)
+    expected = WHOLE_TILE_OUTPUTS[cfg.name]
+    if expected is None:  # uneven blocks: the last tile of a block may be partial
+        expected = sum(r1 - r0 for r0, r1 in ranges) * cfg.hq
+    assert n == expected, (cfg.name, n, expected)
+
+
 def test_fullsize_dense_causal_256k(fullsize_run):
     r = fullsize_run
     cfg = r["cfg"]
@@ -155,6 +208,13 @@ def test_fullsize_dense_causal_256k(fullsize_run):
     do = np.abs(o[rt, ht].float().cpu().numpy() - O_ref).max()
     dl = np.abs(lse[ht, rt].cpu().numpy() - L_ref).max()
     assert do <= O_TOL and dl <= LSE_TOL, (do, dl)
+    # four whole 128-row tiles of the dense kernel, every head: the first, two in the
+    # middle and the last (partial) one
+    last = 128 * ((NT - 1) // 128)
+    ranges = [(0, 128), (100096, 100224), (200064, 200192), (last, NT)]
+    refs = oracle_pool.attention_rows_ranges(r["g"], off, 0, None, 1.0 / math.sqrt(cfg.head_dim), ranges)
+    n = _compare_ranges(o, lse, ranges, refs, "dense 256k")
+    assert n == (3 * 128 + NT - last) * cfg.hq
 
 
 def test_fullsize_two_stage_flow(fullsize_run):

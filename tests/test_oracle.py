@@ -599,3 +599,19 @@ def test_longest_first_within_graham_bound_of_optimum(world, seed):
     best = min(np.bincount(np.array(a), weights=cost, minlength=world).max()
                for a in itertools.product(range(world), repeat=len(cost)))
     assert load.max() <= (4 / 3 - 1 / (3 * world)) * best + 1e-9
+
+
+def test_oracle_pool_matches_direct_calls():
+    """The process pool that full-size GPU tests use for whole-tile comparisons returns
+    exactly what approx_attention gives for the same row ranges."""
+    from . import oracle_pool
+    cfg = CONFIGS["tiny"].with_(n_text=20, n_hosts=4)
+    g = generate(cfg)
+    q, k, v = (orc.bf16_bits_to_f64(g[x]) for x in ("q", "k", "v"))
+    scale = 1 / math.sqrt(cfg.head_dim)
+    full = orc.prefill(q, k, v, g["host_sizes"], cfg.anchor, cfg.passing, cfg.probe_r, scale=scale)
+    ranges = [(0, 128), (256, 384), (384, 512), (512, 532)]
+    res = oracle_pool.attention_rows_ranges(g, full["offsets"], cfg.anchor, full["sel"], scale, ranges, workers=2)
+    for (r0, r1), (O, L) in zip(ranges, res):
+        np.testing.assert_allclose(O, full["O"][r0:r1], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(L, full["lse"][:, r0:r1], rtol=1e-12, atol=1e-12)
