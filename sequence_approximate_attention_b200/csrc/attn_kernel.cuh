@@ -14,8 +14,8 @@
 // forward").
 //
 // CTA = 384 threads, one per SM, persistent over a cost-sorted item list:
-//   warp 0      TMA producer: Q tiles, then K_j, V_j into a ring of smem stages
-//   warp 1      MMA issuer:   S_i = Q_i K_j^T (SS), O_i += P_i V_j (P from TMEM)
+//   warp 0      TMA producer (one thread): Q tiles, then K_j, V_j into a ring of smem stages
+//   warp 1      MMA issuer (one thread): S_i = Q_i K_j^T (SS), O_i += P_i V_j (P from TMEM)
 //   warp 2      TMEM allocator
 //   warps 4-7   softmax of Q tile 0 (TMEM lanes 0..127, one row per thread)
 //   warps 8-11  softmax of Q tile 1
@@ -97,7 +97,10 @@ struct AttnParams {
 // tiles, one softmax warp per 32 rows), every share above 0 was slower: each
 // warp's softmax is bound by its own issue and latency chain, not by MUFU
 // throughput, so the extra instructions cost more than the MUFU time they free.
-constexpr int kPolyPairsOf8 = 0;
+#ifndef SPAVA_POLY_PAIRS_OF_8
+#define SPAVA_POLY_PAIRS_OF_8 0
+#endif
+constexpr int kPolyPairsOf8 = SPAVA_POLY_PAIRS_OF_8;
 
 template <int D>
 struct AttnShape {
@@ -105,7 +108,12 @@ struct AttnShape {
   static constexpr int kHalves = D / 64;            // 128-byte column blocks per row
   static constexpr int kHalfBytes = 128 * 128;      // 128 rows x 128 bytes
   static constexpr int kTileBytes = kHalves * kHalfBytes;
-  static constexpr int kStages = (D == 128) ? 4 : 8;
+#ifndef SPAVA_KV_STAGES_D128
+#define SPAVA_KV_STAGES_D128 5
+#endif
+  // K/V ring stages (K and V tiles alternate); Q, the ring and the barriers fill the
+  // 227 KB a CTA may use at D = 128.
+  static constexpr int kStages = (D == 128) ? SPAVA_KV_STAGES_D128 : 8;
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
@@ -186,19 +194,6 @@ __device__ __forceinline__ AttnItem load_item(const AttnItem* items, int idx) {
   return it;
 }
 
-// Wait on a barrier that no timeout or abort may cut short (draining copies in
-// flight before the CTA exits); still bounded.
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
-  const uint64_t t0 = global_timer_ns();
-  for (;;) {
-    if (mbar_test(bar, parity)) return true;
-    if (global_timer_ns() - t0 > w.limit_ns) {
-      atomicOr(w.err_word, kErrWaitDrain);
-      return false;
-    }
-  }
-}
-
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -253,7 +248,8 @@ __global__ void __launch_bounds__(384, 1)
   const int G = gridDim.x, cta = blockIdx.x;
   if (warp < 4) {
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer (lane 0)
+    if (lane == 0) {
     int ring = 0, m = 0, q_issued = 0;
     bool ok = true;
     if (!p.stall_producer) {
@@ -264,17 +260,14 @@ __global__ void __launch_bounds__(384, 1)
         const int kvh = it.q_head / p.group;
         const bool act1 = it.q_rows > 128;
         if (m > 0) {
-          ok = __all_sync(FULL, mbar_wait(q_empty, (m - 1) & 1, wc, kErrWaitRelease));
+          ok = mbar_wait(q_empty, (m - 1) & 1, wc, kErrWaitRelease);
           if (!ok) break;
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(q_full, (act1 ? 2 : 1) * S::kTileBytes);
-          for (int i = 0; i < (act1 ? 2 : 1); ++i)
-            for (int hh = 0; hh < S::kHalves; ++hh)
-              tma_load_3d(sQ + i * S::kTileBytes + hh * S::kHalfBytes, &tmQ, q_full, hh * 64, it.q_head,
-                          it.q_row0 + i * 128);
-        }
-        __syncwarp();
+        mbar_arrive_expect_tx(q_full, (act1 ? 2 : 1) * S::kTileBytes);
+        for (int i = 0; i < (act1 ? 2 : 1); ++i)
+          for (int hh = 0; hh < S::kHalves; ++hh)
+            tma_load_3d(sQ + i * S::kTileBytes + hh * S::kHalfBytes, &tmQ, q_full, hh * 64, it.q_head,
+                        it.q_row0 + i * 128);
         q_issued = m + 1;
         TileCursor cur;
         for (cur.start(it); !cur.done() && ok; cur.next(it)) {
@@ -284,22 +277,19 @@ __global__ void __launch_bounds__(384, 1)
           for (int kv = 0; kv < 2; ++kv) {
             const int slot = ring % S::kStages, use = ring / S::kStages;
             if (use > 0) {
-              ok = __all_sync(FULL, mbar_wait(kv_empty + slot, (use - 1) & 1, wc, kErrWaitRelease));
+              ok = mbar_wait(kv_empty + slot, (use - 1) & 1, wc, kErrWaitRelease);
               if (!ok) break;
             }
-            if (lane == 0) {
-              uint8_t* dst = sKV + slot * S::kTileBytes;
-              mbar_arrive_expect_tx(kv_full + slot, S::kTileBytes);
-              const CUtensorMap* map = passing ? (kv ? &tmVp : &tmKp) : (kv ? &tmV : &tmK);
-              for (int hh = 0; hh < S::kHalves; ++hh) {
-                if (passing)
-                  tma_load_3d(dst + hh * S::kHalfBytes, map, kv_full + slot, hh * 64, row,
-                              p.pass_per_qhead ? it.q_head : kvh);
-                else
-                  tma_load_3d(dst + hh * S::kHalfBytes, map, kv_full + slot, hh * 64, kvh, row);
-              }
+            uint8_t* dst = sKV + slot * S::kTileBytes;
+            mbar_arrive_expect_tx(kv_full + slot, S::kTileBytes);
+            const CUtensorMap* map = passing ? (kv ? &tmVp : &tmKp) : (kv ? &tmV : &tmK);
+            for (int hh = 0; hh < S::kHalves; ++hh) {
+              if (passing)
+                tma_load_3d(dst + hh * S::kHalfBytes, map, kv_full + slot, hh * 64, row,
+                            p.pass_per_qhead ? it.q_head : kvh);
+              else
+                tma_load_3d(dst + hh * S::kHalfBytes, map, kv_full + slot, hh * 64, kvh, row);
             }
-            __syncwarp();
             ++ring;
           }
         }
@@ -307,18 +297,21 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     if (!ok) {
-      // Abort: let every copy this warp issued land before the CTA exits.
-      if (lane == 0) {
-        for (int s = 0; s < S::kStages; ++s) {
-          const int uses = ring / S::kStages + (s < ring % S::kStages ? 1 : 0);
-          if (uses > 0) mbar_wait_drain(kv_full + s, (uses - 1) & 1, wc);
-        }
-        if (q_issued > 0) mbar_wait_drain(q_full, (q_issued - 1) & 1, wc);
+      // Abort: let every copy this thread issued land before the CTA exits.
+      for (int s = 0; s < S::kStages; ++s) {
+        const int uses = ring / S::kStages + (s < ring % S::kStages ? 1 : 0);
+        if (uses > 0) mbar_wait_drain(kv_full + s, (uses - 1) & 1, wc);
       }
-      __syncwarp();
+      if (q_issued > 0) mbar_wait_drain(q_full, (q_issued - 1) & 1, wc);
     }
+    }
+    __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ MMA issuer (lane 0)
+    // One thread issues every MMA: tcgen05.mma returns only once the tensor core has
+    // taken the instruction, so this thread's issue stream is the tensor core's
+    // schedule and any warp-wide vote or reconvergence in it is idle tensor time.
+    if (lane == 0) {
     int ring = 0, m = 0;
     uint32_t pc0 = 0, pc1 = 0;
     bool ok = true, issued_any = false;
@@ -354,75 +347,63 @@ __global__ void __launch_bounds__(384, 1)
       const AttnItem it = load_item(p.items, idx);
       const int nt = attn_num_tiles(it);
       const bool act1 = it.q_rows > 128;
-      ok = __all_sync(FULL, mbar_wait(q_full, m & 1, wc, kErrWaitLoad));
+      ok = mbar_wait(q_full, m & 1, wc, kErrWaitLoad);
       if (!ok) break;
       int slotK = ring % S::kStages;
-      ok = __all_sync(FULL, mbar_wait(kv_full + slotK, (ring / S::kStages) & 1, wc, kErrWaitLoad));
+      ok = mbar_wait(kv_full + slotK, (ring / S::kStages) & 1, wc, kErrWaitLoad);
       if (!ok) break;
       ++ring;
       tc_fence_after();
-      if (lane == 0) {
-        issue_s(0, slotK);
-        mma_commit(s_full + 0);
-        if (act1) {
-          issue_s(1, slotK);
-          mma_commit(s_full + 1);
-        }
-        mma_commit(kv_empty + slotK);
-        if (nt == 1) mma_commit(q_empty);
+      issue_s(0, slotK);
+      mma_commit(s_full + 0);
+      if (act1) {
+        issue_s(1, slotK);
+        mma_commit(s_full + 1);
       }
+      mma_commit(kv_empty + slotK);
+      if (nt == 1) mma_commit(q_empty);
       issued_any = true;
-      __syncwarp();
       for (int j = 0; j < nt; ++j) {
         const int slotV = ring % S::kStages;
-        ok = __all_sync(FULL, mbar_wait(kv_full + slotV, (ring / S::kStages) & 1, wc, kErrWaitLoad));
+        ok = mbar_wait(kv_full + slotV, (ring / S::kStages) & 1, wc, kErrWaitLoad);
         if (!ok) break;
         ++ring;
-        ok = __all_sync(FULL, mbar_wait(p_full + 0, pc0 & 1, wc, kErrWaitSoftmax));
-        ++pc0;
-        if (!ok) break;
-        tc_fence_after();
-        if (lane == 0) {
-          issue_pv(0, slotV, j > 0);
-          if (j == nt - 1) mma_commit(o_full + 0);
-        }
-        __syncwarp();
+        // K_{j+1} is waited for before P_0(j): the loads run ahead, and this keeps the
+        // wait off the path from the softmax's hand-over to S_0(j+1).
         int slotK2 = -1;
         if (j + 1 < nt) {
           slotK2 = ring % S::kStages;
-          ok = __all_sync(FULL, mbar_wait(kv_full + slotK2, (ring / S::kStages) & 1, wc, kErrWaitLoad));
+          ok = mbar_wait(kv_full + slotK2, (ring / S::kStages) & 1, wc, kErrWaitLoad);
           if (!ok) break;
           ++ring;
-          tc_fence_after();
-          if (lane == 0) {
-            issue_s(0, slotK2);
-            mma_commit(s_full + 0);
-          }
-          __syncwarp();
+        }
+        ok = mbar_wait(p_full + 0, pc0 & 1, wc, kErrWaitSoftmax);
+        ++pc0;
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, slotV, j > 0);
+        if (j == nt - 1) mma_commit(o_full + 0);
+        if (j + 1 < nt) {
+          issue_s(0, slotK2);
+          mma_commit(s_full + 0);
         }
         if (act1) {
-          ok = __all_sync(FULL, mbar_wait(p_full + 1, pc1 & 1, wc, kErrWaitSoftmax));
+          ok = mbar_wait(p_full + 1, pc1 & 1, wc, kErrWaitSoftmax);
           ++pc1;
           if (!ok) break;
           tc_fence_after();
-          if (lane == 0) {
-            issue_pv(1, slotV, j > 0);
-            if (j == nt - 1) mma_commit(o_full + 1);
-            if (j + 1 < nt) {
-              issue_s(1, slotK2);
-              mma_commit(s_full + 1);
-            }
-          }
-          __syncwarp();
-        }
-        if (lane == 0) {
-          mma_commit(kv_empty + slotV);
+          issue_pv(1, slotV, j > 0);
+          if (j == nt - 1) mma_commit(o_full + 1);
           if (j + 1 < nt) {
-            mma_commit(kv_empty + slotK2);
-            if (j + 1 == nt - 1) mma_commit(q_empty);
+            issue_s(1, slotK2);
+            mma_commit(s_full + 1);
           }
         }
-        __syncwarp();
+        mma_commit(kv_empty + slotV);
+        if (j + 1 < nt) {
+          mma_commit(kv_empty + slotK2);
+          if (j + 1 == nt - 1) mma_commit(q_empty);
+        }
       }
       if (!ok) break;
       ++m;
@@ -431,12 +412,11 @@ __global__ void __launch_bounds__(384, 1)
       // Every MMA issued so far must finish before TMEM is released (on the normal
       // path the softmax warps have already seen them finish; after an abort they
       // may still be running).
-      if (lane == 0) {
-        mma_commit(drain);
-        mbar_wait_drain(drain, 0, wc);
-      }
-      __syncwarp();
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0, wc);
     }
+    }
+    __syncwarp();
   }
   } else {
     // ------------------------------------------------------------ softmax / epilogue

@@ -18,8 +18,8 @@
 // of Rc probe tokens (Rc G <= 256).  Work item = one 128-key tile of one (host, KV
 // head).
 //
-// CTA = 256 threads: warp 0 TMA, warp 1 MMA, warp 2 TMEM allocator,
-// warps 4-7 epilogue (lane = key).  TMEM holds two 256-column accumulators so the
+// CTA = 256 threads: warp 0 TMA (one thread), warp 1 MMA (one thread), warp 2 TMEM
+// allocator, warps 4-7 epilogue (lane = key).  TMEM holds two 256-column accumulators so the
 // epilogue of one chunk overlaps the MMA of the next.
 #pragma once
 
@@ -153,47 +153,35 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    int qloads[2] = {0, 0};
-    int slot = 0, use = 0;  // K stage and how often it was filled before (no division)
-    bool ok = true;
-    for (int li = 0; li < n_local && ok; ++li) {
-      const int4 it = s_items[li];
-      if (use > 0) {
-        ok = __all_sync(FULL, mbar_wait(k_empty + slot, (use - 1) & 1, wc, kErrWaitRelease));
-        if (!ok) break;
-      }
-      if (lane == 0) {
+    // ------------------------------------------------------------ TMA producer (lane 0)
+    if (lane == 0) {
+      int qloads[2] = {0, 0};
+      int slot = 0, use = 0;  // K stage and how often it was filled before (no division)
+      bool ok = true;
+      for (int li = 0; li < n_local && ok; ++li) {
+        const int4 it = s_items[li];
+        if (use > 0 && !(ok = mbar_wait(k_empty + slot, (use - 1) & 1, wc, kErrWaitRelease))) break;
         mbar_arrive_expect_tx(k_full + slot, S::kKTileBytes);
         for (int hh = 0; hh < S::kHalves; ++hh)
           tma_load_3d(sK + slot * S::kKTileBytes + hh * 128 * 128, &tmK, k_full + slot, hh * 64, it.y, it.z);
-      }
-      __syncwarp();
-      if (++slot == n_stages) {
-        slot = 0;
-        ++use;
-      }
-      for (int c = 0; c < p.n_chunks; ++c) {
-        const int u = li * p.n_chunks + c, b = u & (p.q_bufs - 1);
-        if (!score_needs_load(p, s_items, li, c)) continue;
-        if (qloads[b] > 0) {
-          ok = __all_sync(FULL, mbar_wait(q_empty + b, (qloads[b] - 1) & 1, wc, kErrWaitRelease));
-          if (!ok) break;
+        if (++slot == n_stages) {
+          slot = 0;
+          ++use;
         }
-        if (lane == 0) {
+        for (int c = 0; c < p.n_chunks; ++c) {
+          const int u = li * p.n_chunks + c, b = u & (p.q_bufs - 1);
+          if (!score_needs_load(p, s_items, li, c)) continue;
+          if (qloads[b] > 0 && !(ok = mbar_wait(q_empty + b, (qloads[b] - 1) & 1, wc, kErrWaitRelease))) break;
           mbar_arrive_expect_tx(q_full + b, static_cast<uint32_t>(S::kHalves * p.chunk_tokens * G * 128));
           for (int hh = 0; hh < S::kHalves; ++hh)
             for (int h = 0; h < G; ++h)
               tma_load_3d(sQ + b * p.q_buf_bytes + hh * (p.chunk_tokens * G * 128) + h * (p.chunk_tokens * 128), &tmQp,
                           q_full + b, hh * 64, it.y * G + h, it.w - p.probe_r + c * p.chunk_tokens);
+          ++qloads[b];
         }
-        __syncwarp();
-        ++qloads[b];
       }
-    }
-    if (!ok) {
-      // Abort: let every copy this warp issued land before the CTA exits.
-      if (lane == 0) {
+      if (!ok) {
+        // Abort: let every copy this thread issued land before the CTA exits.
         for (int b = 0; b < n_stages; ++b) {
           const int uses = use + (b < slot ? 1 : 0);  // loads issued into stage b
           if (uses > 0) mbar_wait_drain(k_full + b, (uses - 1) & 1, wc);
@@ -201,34 +189,32 @@ __global__ void __launch_bounds__(256, 1)
         for (int b = 0; b < 2; ++b)
           if (qloads[b] > 0) mbar_wait_drain(q_full + b, (qloads[b] - 1) & 1, wc);
       }
-      __syncwarp();
     }
+    __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    int qloads[2] = {0, 0};
-    bool ok = true, issued_any = false;
-    int slot = 0, kphase = 0;
-    for (int li = 0; li < n_local && ok; ++li) {
-      ok = __all_sync(FULL, mbar_wait(k_full + slot, kphase, wc, kErrWaitLoad));
-      if (!ok) break;
-      for (int c = 0; c < p.n_chunks; ++c) {
-        const int u = li * p.n_chunks + c;
-        const int qb = u & (p.q_bufs - 1);  // probe-query buffer (q_bufs is 1 or 2)
-        const int ab = u & 1;               // TMEM accumulator
-        if (score_needs_load(p, s_items, li, c)) {
-          ok = __all_sync(FULL, mbar_wait(q_full + qb, qloads[qb] & 1, wc, kErrWaitLoad));
-          ++qloads[qb];
-          if (!ok) break;
-        }
-        if (u >= 2) {
-          ok = __all_sync(FULL, mbar_wait(acc_empty + ab, ((u >> 1) - 1) & 1, wc, kErrWaitMma));
-          if (!ok) break;
-        }
-        tc_fence_after();
-        // All Rc G columns: with (head, token) order a short last chunk's probe rows
-        // are not a prefix; the epilogue masks the rest.
-        const int nc = p.chunk_tokens * G;
-        if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (lane 0)
+    // One thread issues every MMA (tcgen05.mma returns once the tensor core has taken
+    // the instruction), with no warp-wide votes between them.
+    if (lane == 0) {
+      int qloads[2] = {0, 0};
+      bool ok = true, issued_any = false;
+      int slot = 0, kphase = 0;
+      for (int li = 0; li < n_local && ok; ++li) {
+        if (!(ok = mbar_wait(k_full + slot, kphase, wc, kErrWaitLoad))) break;
+        for (int c = 0; c < p.n_chunks; ++c) {
+          const int u = li * p.n_chunks + c;
+          const int qb = u & (p.q_bufs - 1);  // probe-query buffer (q_bufs is 1 or 2)
+          const int ab = u & 1;               // TMEM accumulator
+          if (score_needs_load(p, s_items, li, c)) {
+            ok = mbar_wait(q_full + qb, qloads[qb] & 1, wc, kErrWaitLoad);
+            ++qloads[qb];
+            if (!ok) break;
+          }
+          if (u >= 2 && !(ok = mbar_wait(acc_empty + ab, ((u >> 1) - 1) & 1, wc, kErrWaitMma))) break;
+          tc_fence_after();
+          // All Rc G columns: with (head, token) order a short last chunk's probe rows
+          // are not a prefix; the epilogue masks the rest.
+          const int nc = p.chunk_tokens * G;
           const uint32_t idesc = idesc_bf16_f32(128, nc, 0, 0);
           const uint32_t ka = smem_u32(sK + slot * S::kKTileBytes);
           const uint32_t qa = smem_u32(sQ + qb * p.q_buf_bytes);
@@ -243,25 +229,21 @@ __global__ void __launch_bounds__(256, 1)
           int ln, cn;
           score_next_use(p, li, c, &ln, &cn);
           if (ln < n_local && score_needs_load(p, s_items, ln, cn)) mma_commit(q_empty + qb);
+          issued_any = true;
         }
-        issued_any = true;
-        __syncwarp();
+        if (!ok) break;
+        mma_commit(k_empty + slot);
+        if (++slot == n_stages) {
+          slot = 0;
+          kphase ^= 1;
+        }
       }
-      if (!ok) break;
-      if (lane == 0) mma_commit(k_empty + slot);
-      __syncwarp();
-      if (++slot == n_stages) {
-        slot = 0;
-        kphase ^= 1;
-      }
-    }
-    if (issued_any) {
-      if (lane == 0) {
+      if (issued_any) {
         mma_commit(drain);
         mbar_wait_drain(drain, 0, wc);
       }
-      __syncwarp();
     }
+    __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue: one key per thread
     const int qd = warp & 3;

@@ -27,7 +27,7 @@ def test_tmem_wrappers_cover_the_widths_in_use():
     used = set()
     for name in os.listdir(CSRC):
         if name.endswith((".cuh", ".cu")):
-            used |= set(re.findall(r"tmem_(ld|st)_x(\d+)\(", open(os.path.join(CSRC, name)).read()))
-    for kind, n in used:
-        widths = gen.LOAD_WIDTHS if kind == "ld" else gen.STORE_WIDTHS
-        assert int(n) in widths, (kind, n)
+            used |= set(re.findall(r"tmem_(ld|st)_x(\d+)(_async)?\(", open(os.path.join(CSRC, name)).read()))
+    for kind, n, asy in used:
+        widths = gen.ASYNC_STORE_WIDTHS if asy else gen.LOAD_WIDTHS if kind == "ld" else gen.STORE_WIDTHS
+        assert int(n) in widths, (kind, n, asy)
