@@ -785,11 +785,36 @@ def main():
             t1.record(stream)
             torch.cuda.synchronize(dev)
             times["dense" if dense_mode else "approx"] = max_over_ranks(t0.elapsed_time(t1), dev) / 2
+        stack.check_errors()
+        # the projection kernels alone: one layer's QKV projection (RMSNorm fused) and
+        # output projection + residual, timed on the stack's own buffers
+        L0 = stack.layers[0]
+        sab.qkv_projection(stack._x, L0["w_qkv"], cfg.hq, cfg.hkv, cfg.head_dim, stack._q, stack._k, stack._v,
+                           stack.ws_layer)
+        reps = 5
+        t0, t1, t2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        t0.record(stream)
+        for _ in range(reps):
+            sab.qkv_projection(stack._x, L0["w_qkv"], cfg.hq, cfg.hkv, cfg.head_dim, stack._q, stack._k, stack._v,
+                               stack.ws_layer)
+        t1.record(stream)
+        for _ in range(reps):
+            sab.out_projection(stack._o, L0["w_o"], stack._x, stack.ws_layer)
+        t2.record(stream)
+        torch.cuda.synchronize(dev)
+        stack.check_errors()
+        fl = stack.flops()
+        qkv_ms, out_ms = t0.elapsed_time(t1) / reps, t1.elapsed_time(t2) / reps
         ttft = {"layers": args.ttft_layers, "hidden": hidden, "tokens": NT, "approx_ms": times["approx"],
                 "dense_ms": times["dense"], "speedup": times["dense"] / times["approx"],
-                "projection_tflop_per_layer": stack.flops()["projections"] / 1e12,
-                "note": "attention blocks only (RMSNorm, QKV and output projections, attention, residual); "
-                        "random weights, no rotary embedding, no MLP"}
+                "projection_tflop_per_layer": fl["projections"] / 1e12,
+                "qkv_projection": {"ms": qkv_ms, "TFLOP/s": fl["qkv"] / (qkv_ms / 1e3) / 1e12,
+                                   "frac": fl["qkv"] / (qkv_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
+                "out_projection": {"ms": out_ms, "TFLOP/s": fl["out"] / (out_ms / 1e3) / 1e12,
+                                   "frac": fl["out"] / (out_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
+                "note": "attention blocks only: RMSNorm + QKV projection (tcgen05 GEMM, norm and q/k/v split "
+                        "in its epilogue), attention, output projection + residual (tcgen05 GEMM); random "
+                        "weights, no rotary embedding, no MLP"}
         del stack
 
     cpu = None

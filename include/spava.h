@@ -424,6 +424,52 @@ spava_status spava_profile_end(spava_plan* plan);
  * 12 spare text-slot fill (sharded prefill). */
 const char* spava_kernel_name(int32_t label);
 
+/*
+ * The linear maps around the attention of one decoder layer, for a multi-layer
+ * prefill (the pages report time to first token: APB-V technical summary,
+ * "Experimental results"; their fused forward of context and query runs every token
+ * of the layer through the same projections, 2. System optimisations, "Fused context
+ * and query forward").  Both run a tcgen05 GEMM (TMA-fed, TMEM accumulators, 128 x
+ * 256 output tiles, persistent over the SMs) with a fused epilogue.  Pointers are
+ * device pointers owned by the caller; bf16 tensors are row-major with the last
+ * dimension contiguous; all must be 16-byte aligned.  Calls are asynchronous on
+ * `stream` and allocate nothing.
+ *
+ * spava_layer_workspace_bytes(n_tokens): bytes of the caller's workspace `ws`
+ * (256-byte aligned) that both calls of a layer use: a device error word and the
+ * rows' RMS factors.  Returns 0 for n_tokens < 0.
+ *
+ * spava_qkv_projection: RMSNorm + QKV projection.
+ *   x      [n_tokens][hidden] bf16, the layer's input hidden states;
+ *   w_qkv  [(hq + 2 hkv) head_dim][hidden] bf16: the query, key and value weights
+ *          stacked row-wise (row j of the stack produces output feature j);
+ *   q      [n_tokens][hq][head_dim], k and v [n_tokens][hkv][head_dim] bf16 (the
+ *          layouts spava_attn_prefill reads), written:
+ *            y = (x / rms(x)) W_qkv^T,  rms(x_m) = sqrt(mean_j x_mj^2 + rms_eps),
+ *          columns [0, hq d) of y into q, [hq d, (hq + hkv) d) into k, the rest into v.
+ *   The row scale 1 / rms is applied to the fp32 accumulator (the normalised x is
+ *   never stored); outputs are rounded to bf16 (RNE).  Clears the workspace error word.
+ *   Errors: SPAVA_ERR_INVALID_ARG for NULL or misaligned pointers, non-positive sizes,
+ *   hq % hkv != 0 or rms_eps <= 0; SPAVA_ERR_UNSUPPORTED unless hidden, hq head_dim
+ *   and hkv head_dim are multiples of 256 or when the device is not sm_100.
+ *
+ * spava_out_projection: output projection + residual, in place:
+ *   x[m][:] += o[m][:] W_o^T,  o [n_tokens][in_features] bf16 (the attention output,
+ *   [n_tokens][hq][head_dim] read as rows of hq head_dim), w_o [hidden][in_features]
+ *   bf16, x [n_tokens][hidden] bf16 (read, then overwritten with the rounded sum).
+ *   Errors as above; in_features and hidden must be multiples of 256.
+ *
+ * spava_layer_check_error: synchronise `stream`, read and clear the workspace error
+ *   word; SPAVA_ERR_TIMEOUT if a bounded device wait of either call ran out.
+ */
+size_t spava_layer_workspace_bytes(int32_t n_tokens);
+spava_status spava_qkv_projection(const void* x, int32_t n_tokens, int32_t hidden, const void* w_qkv, int32_t hq,
+                                  int32_t hkv, int32_t head_dim, float rms_eps, void* q, void* k, void* v, void* ws,
+                                  void* stream);
+spava_status spava_out_projection(const void* o, int32_t n_tokens, int32_t in_features, const void* w_o,
+                                  int32_t hidden, void* x, void* ws, void* stream);
+spava_status spava_layer_check_error(void* ws, void* stream);
+
 /* Static text of a status code. */
 const char* spava_status_string(spava_status status);
 

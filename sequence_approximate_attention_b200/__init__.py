@@ -19,7 +19,8 @@ from . import _lib
 from ._lib import SpavaError, load  # noqa: F401
 
 __all__ = ["Plan", "score_select", "gather_passing", "attn_prefill", "attn_prefill_two_stage", "dense_causal",
-           "check_device_error", "SpavaError", "load", "last_launch_count", "shard_owners", "shard_stage"]
+           "check_device_error", "SpavaError", "load", "last_launch_count", "shard_owners", "shard_stage",
+           "layer_workspace", "qkv_projection", "out_projection", "check_layer_error"]
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -375,3 +376,59 @@ def check_device_error(plan: Plan, workspace: torch.Tensor, stream=None) -> None
 
 def last_launch_count() -> int:
     return int(_lib.load().spava_last_launch_count())
+
+
+# ---------------------------------------------------------------- layer projections
+def layer_workspace(n_tokens: int, device=None) -> torch.Tensor:
+    """Workspace of spava_qkv_projection / spava_out_projection for n_tokens rows."""
+    n = int(_lib.load().spava_layer_workspace_bytes(int(n_tokens)))
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=dev)
+
+
+def _check_layer_ws(ws: torch.Tensor, n_tokens: int, device) -> None:
+    need = int(_lib.load().spava_layer_workspace_bytes(int(n_tokens)))
+    if ws.dtype != torch.uint8 or ws.numel() < need or ws.device != device or ws.data_ptr() % 256:
+        raise ValueError(f"layer workspace: uint8, 256-byte aligned, >= {need} bytes on {device}")
+
+
+def qkv_projection(x: torch.Tensor, w_qkv: torch.Tensor, hq: int, hkv: int, head_dim: int,
+                   q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, workspace: torch.Tensor,
+                   rms_eps: float = 1e-6, stream=None) -> None:
+    """q, k, v = split((x / rms(x)) w_qkv^T) on the tensor cores (spava_qkv_projection).
+    x [T, hidden], w_qkv [(hq + 2 hkv) head_dim, hidden], q [T, hq, head_dim],
+    k/v [T, hkv, head_dim]: bf16, contiguous, on one device."""
+    if x.dim() != 2:
+        raise ValueError("x must be [tokens, hidden]")
+    T, hidden = x.shape
+    dev = x.device
+    _expect(x, "x", torch.bfloat16, (T, hidden), dev)
+    _expect(w_qkv, "w_qkv", torch.bfloat16, ((hq + 2 * hkv) * head_dim, hidden), dev)
+    _expect(q, "q", torch.bfloat16, (T, hq, head_dim), dev)
+    _expect(k, "k", torch.bfloat16, (T, hkv, head_dim), dev)
+    _expect(v, "v", torch.bfloat16, (T, hkv, head_dim), dev)
+    _check_layer_ws(workspace, T, dev)
+    st = _lib.load().spava_qkv_projection(_ptr(x), T, hidden, _ptr(w_qkv), hq, hkv, head_dim, float(rms_eps),
+                                          _ptr(q), _ptr(k), _ptr(v), _ptr(workspace), _stream(stream))
+    _lib.check(st, "spava_qkv_projection")
+
+
+def out_projection(o: torch.Tensor, w_o: torch.Tensor, x: torch.Tensor, workspace: torch.Tensor,
+                   stream=None) -> None:
+    """x += o w_o^T in place on the tensor cores (spava_out_projection).  o [T, ...]
+    read as [T, in_features], w_o [hidden, in_features], x [T, hidden]: bf16."""
+    T, hidden = x.shape
+    dev = x.device
+    in_features = o.numel() // max(T, 1)
+    _expect(o.view(T, in_features), "o", torch.bfloat16, (T, in_features), dev)
+    _expect(w_o, "w_o", torch.bfloat16, (hidden, in_features), dev)
+    _expect(x, "x", torch.bfloat16, (T, hidden), dev)
+    _check_layer_ws(workspace, T, dev)
+    st = _lib.load().spava_out_projection(_ptr(o), T, in_features, _ptr(w_o), hidden, _ptr(x), _ptr(workspace),
+                                          _stream(stream))
+    _lib.check(st, "spava_out_projection")
+
+
+def check_layer_error(workspace: torch.Tensor, stream=None) -> None:
+    """Synchronise and raise SpavaError(SPAVA_ERR_TIMEOUT) if a projection's bounded wait ran out."""
+    _lib.check(_lib.load().spava_layer_check_error(_ptr(workspace), _stream(stream)), "spava_layer_check_error")

@@ -75,6 +75,12 @@ SIGNATURES = {
                                      c_int32]),
     "spava_profile_end": (c_int32, [c_void_p]),
     "spava_kernel_name": (ctypes.c_char_p, [c_int32]),
+    "spava_layer_workspace_bytes": (c_size_t, [c_int32]),
+    "spava_qkv_projection": (c_int32, [c_void_p, c_int32, c_int32, c_void_p, c_int32, c_int32, c_int32,
+                                       ctypes.c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "spava_out_projection": (c_int32, [c_void_p, c_int32, c_int32, c_void_p, c_int32, c_void_p, c_void_p,
+                                       c_void_p]),
+    "spava_layer_check_error": (c_int32, [c_void_p, c_void_p]),
 }
 
 _LIB = None

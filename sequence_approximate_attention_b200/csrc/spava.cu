@@ -24,6 +24,7 @@
 
 #include "attn_kernel.cuh"
 #include "common.cuh"
+#include "proj_kernel.cuh"
 #include "score_kernel.cuh"
 #include "select_gather.cuh"
 
@@ -89,6 +90,22 @@ spava_status make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t 
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SPAVA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return SPAVA_OK;
+}
+
+// 2-D bf16 tensor map with 128-byte swizzle over a row-major [outer][inner] matrix
+// (inner contiguous); box (64, box_outer); rows past `outer` read as zero.
+spava_status make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return fail(SPAVA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {64, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SPAVA_ERR_CUDA, "cuTensorMapEncodeTiled (2-D) failed (%d)", static_cast<int>(r));
   return SPAVA_OK;
 }
 
@@ -1402,6 +1419,131 @@ spava_status spava_check_device_error(const spava_plan* p, void* ws, void* strea
     SPAVA_CUDA(cudaMemsetAsync(err_word(p, ws), 0, 256, st));
     SPAVA_CUDA(cudaStreamSynchronize(st));
     return fail(SPAVA_ERR_TIMEOUT, "a bounded device wait ran out (error bits 0x%x)", word);
+  }
+  return ok();
+}
+
+}  // extern "C"
+
+// =================================================================== layer projections
+namespace {
+
+constexpr size_t kLayerErrBytes = 256;
+
+// Current device, checked to be an sm_100 part; its SM count.
+spava_status layer_device(int* num_sms) {
+  int dev = -1, major = 0, minor = 0;
+  SPAVA_CUDA(cudaGetDevice(&dev));
+  SPAVA_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  SPAVA_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+  if (major != 10 || minor != 0)
+    return fail(SPAVA_ERR_UNSUPPORTED, "needs an sm_100 (B200) device, found sm_%d%d", major, minor);
+  SPAVA_CUDA(cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev));
+  return SPAVA_OK;
+}
+
+spava_status launch_proj(const void* a, int M, int K, const void* w, int N, spava::ProjParams pp, int num_sms,
+                         cudaStream_t st) {
+  using S = spava::ProjShape;
+  CUtensorMap tmA, tmB;
+  spava_status s;
+  if ((s = make_map_2d(&tmA, a, K, M, S::kBM)) != SPAVA_OK) return s;
+  if ((s = make_map_2d(&tmB, w, K, N, S::kBN)) != SPAVA_OK) return s;
+  pp.M = M;
+  pp.K = K;
+  pp.N = N;
+  pp.n_tiles_n = N / S::kBN;
+  pp.n_tiles = ceil_div(M, S::kBM) * pp.n_tiles_n;
+  pp.wait_limit_ns = spava::kDefaultWaitLimitNs;
+  if ((s = ensure_smem(spava::proj_gemm_kernel, S::kSmemBytes)) != SPAVA_OK) return s;
+  spava::proj_gemm_kernel<<<std::min(pp.n_tiles, num_sms), S::kThreads, S::kSmemBytes, st>>>(tmA, tmB, pp);
+  SPAVA_CUDA(cudaGetLastError());
+  ++g_last_launches;
+  return SPAVA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t spava_layer_workspace_bytes(int32_t n_tokens) {
+  return n_tokens < 0 ? 0 : kLayerErrBytes + align_up(static_cast<size_t>(n_tokens) * 4, 256);
+}
+
+spava_status spava_qkv_projection(const void* x, int32_t n_tokens, int32_t hidden, const void* w_qkv, int32_t hq,
+                                  int32_t hkv, int32_t head_dim, float rms_eps, void* q, void* k, void* v, void* ws,
+                                  void* stream) {
+  g_last_launches = 0;
+  if (!x || !w_qkv || !q || !k || !v || !ws) return fail(SPAVA_ERR_INVALID_ARG, "NULL pointer");
+  if (n_tokens < 1 || hidden < 1 || hq < 1 || hkv < 1 || head_dim < 1 || hq % hkv)
+    return fail(SPAVA_ERR_INVALID_ARG, "need n_tokens, hidden, hq, hkv, head_dim >= 1 and hq %% hkv == 0");
+  if (!(rms_eps > 0.f)) return fail(SPAVA_ERR_INVALID_ARG, "rms_eps must be positive");
+  const int nq = hq * head_dim, nk = hkv * head_dim;
+  if (hidden % 256 || nq % 256 || nk % 256)
+    return fail(SPAVA_ERR_UNSUPPORTED, "hidden, hq * head_dim and hkv * head_dim must be multiples of 256");
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q) || !aligned16(k) || !aligned16(v))
+    return fail(SPAVA_ERR_INVALID_ARG, "x, w_qkv, q, k, v must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(SPAVA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  int num_sms = 0;
+  spava_status s;
+  if ((s = layer_device(&num_sms)) != SPAVA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  float* inv_rms = reinterpret_cast<float*>(w8 + kLayerErrBytes);
+  SPAVA_CUDA(cudaMemsetAsync(w8, 0, kLayerErrBytes, st));
+  spava::rms_rows_kernel<<<ceil_div(n_tokens, 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), n_tokens,
+                                                                 hidden, rms_eps, inv_rms);
+  SPAVA_CUDA(cudaGetLastError());
+  ++g_last_launches;
+  spava::ProjParams pp;
+  std::memset(&pp, 0, sizeof(pp));
+  pp.mode = spava::kProjQKV;
+  pp.nq = nq;
+  pp.nk = nk;
+  pp.q = static_cast<__nv_bfloat16*>(q);
+  pp.k = static_cast<__nv_bfloat16*>(k);
+  pp.v = static_cast<__nv_bfloat16*>(v);
+  pp.inv_rms = inv_rms;
+  pp.err_word = reinterpret_cast<unsigned int*>(w8);
+  if ((s = launch_proj(x, n_tokens, hidden, w_qkv, nq + 2 * nk, pp, num_sms, st)) != SPAVA_OK) return s;
+  return ok();
+}
+
+spava_status spava_out_projection(const void* o, int32_t n_tokens, int32_t in_features, const void* w_o,
+                                  int32_t hidden, void* x, void* ws, void* stream) {
+  g_last_launches = 0;
+  if (!o || !w_o || !x || !ws) return fail(SPAVA_ERR_INVALID_ARG, "NULL pointer");
+  if (n_tokens < 1 || in_features < 1 || hidden < 1) return fail(SPAVA_ERR_INVALID_ARG, "sizes must be positive");
+  if (in_features % 256 || hidden % 256)
+    return fail(SPAVA_ERR_UNSUPPORTED, "in_features and hidden must be multiples of 256");
+  if (!aligned16(o) || !aligned16(w_o) || !aligned16(x))
+    return fail(SPAVA_ERR_INVALID_ARG, "o, w_o, x must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(SPAVA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  int num_sms = 0;
+  spava_status s;
+  if ((s = layer_device(&num_sms)) != SPAVA_OK) return s;
+  spava::ProjParams pp;
+  std::memset(&pp, 0, sizeof(pp));
+  pp.mode = spava::kProjResidual;
+  pp.residual = static_cast<const __nv_bfloat16*>(x);
+  pp.out = static_cast<__nv_bfloat16*>(x);
+  pp.err_word = static_cast<unsigned int*>(ws);
+  if ((s = launch_proj(o, n_tokens, in_features, w_o, hidden, pp, num_sms, static_cast<cudaStream_t>(stream))) !=
+      SPAVA_OK)
+    return s;
+  return ok();
+}
+
+spava_status spava_layer_check_error(void* ws, void* stream) {
+  if (!ws) return fail(SPAVA_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SPAVA_CUDA(cudaStreamSynchronize(st));
+  unsigned int word = 0;
+  SPAVA_CUDA(cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost));
+  if (word) {
+    SPAVA_CUDA(cudaMemsetAsync(ws, 0, kLayerErrBytes, st));
+    SPAVA_CUDA(cudaStreamSynchronize(st));
+    return fail(SPAVA_ERR_TIMEOUT, "a bounded device wait ran out in a projection (error bits 0x%x)", word);
   }
   return ok();
 }
