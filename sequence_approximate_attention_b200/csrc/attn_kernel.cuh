@@ -252,6 +252,11 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
     int ring = 0, m = 0, q_issued = 0;
     bool ok = true;
+#ifndef SPAVA_NO_L2_HINTS
+    // Q tiles are read by one item only; K/V rows (own block, anchor, passing) by the
+    // items of every query head of the group and every later row block.
+    const uint64_t pol_q = l2_policy_evict_first(), pol_kv = l2_policy_evict_last();
+#endif
     if (!p.stall_producer) {
       for (int r = 0; ok; ++r) {
         const int idx = attn_sched(r, cta, G);
@@ -265,9 +270,15 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbar_arrive_expect_tx(q_full, (act1 ? 2 : 1) * S::kTileBytes);
         for (int i = 0; i < (act1 ? 2 : 1); ++i)
-          for (int hh = 0; hh < S::kHalves; ++hh)
+          for (int hh = 0; hh < S::kHalves; ++hh) {
+#ifndef SPAVA_NO_L2_HINTS
+            tma_load_3d_hint(sQ + i * S::kTileBytes + hh * S::kHalfBytes, &tmQ, q_full, hh * 64, it.q_head,
+                             it.q_row0 + i * 128, pol_q);
+#else
             tma_load_3d(sQ + i * S::kTileBytes + hh * S::kHalfBytes, &tmQ, q_full, hh * 64, it.q_head,
                         it.q_row0 + i * 128);
+#endif
+          }
         q_issued = m + 1;
         TileCursor cur;
         for (cur.start(it); !cur.done() && ok; cur.next(it)) {
@@ -284,11 +295,19 @@ __global__ void __launch_bounds__(384, 1)
             mbar_arrive_expect_tx(kv_full + slot, S::kTileBytes);
             const CUtensorMap* map = passing ? (kv ? &tmVp : &tmKp) : (kv ? &tmV : &tmK);
             for (int hh = 0; hh < S::kHalves; ++hh) {
+#ifndef SPAVA_NO_L2_HINTS
+              if (passing)
+                tma_load_3d_hint(dst + hh * S::kHalfBytes, map, kv_full + slot, hh * 64, row,
+                                 p.pass_per_qhead ? it.q_head : kvh, pol_kv);
+              else
+                tma_load_3d_hint(dst + hh * S::kHalfBytes, map, kv_full + slot, hh * 64, kvh, row, pol_kv);
+#else
               if (passing)
                 tma_load_3d(dst + hh * S::kHalfBytes, map, kv_full + slot, hh * 64, row,
                             p.pass_per_qhead ? it.q_head : kvh);
               else
                 tma_load_3d(dst + hh * S::kHalfBytes, map, kv_full + slot, hh * 64, kvh, row);
+#endif
             }
             ++ring;
           }

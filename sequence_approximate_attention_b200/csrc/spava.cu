@@ -199,11 +199,13 @@ void sort_by_cost(std::vector<AttnItem>& v) {
   std::stable_sort(v.begin(), v.end(), [](const AttnItem& a, const AttnItem& b) { return item_cost(a) > item_cost(b); });
 }
 
-// Prefill order: hosts from the longest KV list to the shortest, KV groups in order
-// inside a host, longest items first inside a group.  Consecutive items (which run
-// at the same time on the 148 CTAs) then share one host's block, the anchor and the
-// passing rows of one or two KV groups, a working set that stays in L2, while every
-// round of CTAs still gets a spread of item costs for balance.
+// Prefill order: KV groups in order; inside a group, hosts from the longest KV list to
+// the shortest; longest items first inside a (group, host).  Consecutive items (which
+// run at the same time on the 148 CTAs) then share one host's block of one KV head,
+// and every host of a group reads the same anchor and passing rows of that KV head,
+// which therefore stay in L2 from the first host of the group to the last (ordering
+// hosts outermost re-read them from DRAM once per host); every round of CTAs still
+// gets a spread of item costs for balance.
 // `group` gives each item its host (text pieces are grouped with the host block
 // they read, their own causal piece with the last host).
 void sort_host_major(std::vector<AttnItem>& v, const std::vector<int>& group, int heads_per_group) {
@@ -211,8 +213,8 @@ void sort_host_major(std::vector<AttnItem>& v, const std::vector<int>& group, in
   std::vector<int> order(v.size());
   for (size_t i = 0; i < v.size(); ++i) order[i] = static_cast<int>(i);
   std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
-    if (group[a] != group[b]) return group[a] > group[b];
     if (kv_group_of(v[a]) != kv_group_of(v[b])) return kv_group_of(v[a]) < kv_group_of(v[b]);
+    if (group[a] != group[b]) return group[a] > group[b];
     return item_cost(v[a]) > item_cost(v[b]);
   });
   std::vector<AttnItem> out;
