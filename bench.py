@@ -75,7 +75,8 @@ def select_gather_bytes(cfg, sizes):
     score = n_scored * hkv * d * 2 + (H - 1) * R * hq * d * 2 + n_scored * hkv * 4
     select = n_scored * hkv * 4 + (H - 1) * hkv * P * 4
     gather = 2 * 2 * (H - 1) * hkv * P * d * 2 + (H - 1) * hkv * P * 4
-    return {"score": score, "select": select, "gather": gather, "select_gather": select + gather}
+    return {"score": score, "select": select, "gather": gather, "select_gather": select + gather,
+            "score_select_gather": score + select + gather}
 
 
 def attn_algorithmic_bytes(cfg):
@@ -556,6 +557,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="128k", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--fused-select", type=int, default=0,
+                    help="0: score kernel, then select+gather (default); 1: scoring, selection and gather in "
+                         "one persistent launch")
     ap.add_argument("--flow", default="single", choices=["single", "two_stage"],
                     help="single: one attention pass per host (default); two_stage: local pass with fused "
                          "probe scores, then the remote pass merged through the lse")
@@ -622,6 +626,7 @@ def main():
     plan = sab.Plan(cfg.n_visual, cfg.n_text, cfg.n_hosts, sizes, cfg.anchor, cfg.passing, cfg.probe_r,
                     cfg.hq, cfg.hkv, cfg.head_dim, device=dev)
     two_stage = args.flow == "two_stage"
+    plan.set_fused_select(bool(args.fused_select))
     ws = plan.new_workspace(two_stage)
     o = torch.empty_like(d_in["q"])
     prefill = sab.attn_prefill_two_stage if two_stage else sab.attn_prefill
@@ -672,7 +677,7 @@ def main():
     achieved = flops / (avg.get("attention", float("nan")) / 1e3) / 1e12
     sgb = select_gather_bytes(cfg, sizes)
     hbm = {}
-    for name in ("score", "select", "gather", "select_gather"):
+    for name in ("score", "select", "gather", "select_gather", "score_select_gather"):
         if name in avg:
             gbs = sgb[name] / (avg[name] / 1e3) / 1e9
             hbm[name] = {"ms": avg[name], "bytes": sgb[name], "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]}
@@ -682,7 +687,7 @@ def main():
         hbm["score"]["flops"] = sf
         hbm["score"]["TFLOP/s"] = sf / (avg["score"] / 1e3) / 1e12
         hbm["score"]["frac_of_tensor_peak"] = hbm["score"]["TFLOP/s"] / peaks["bf16_tflops"]
-    ssg_names = [n for n in ("score", "select", "gather", "select_gather") if n in avg]
+    ssg_names = [n for n in ("score", "select", "gather", "select_gather", "score_select_gather") if n in avg]
     ssg_ms = sum(avg[n] for n in ssg_names)
     ssg_bytes = sum(sgb[n] for n in ssg_names)
     roofline = {
@@ -828,7 +833,7 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "b200", "flow": args.flow,
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "b200", "flow": args.flow, "fused_select": bool(args.fused_select),
             "config": workload_config(cfg),
             "tflops_step": step_tflops, "tflops_step_frac": step_tflops / peaks["bf16_tflops"],
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "ttft": ttft,

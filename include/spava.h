@@ -145,6 +145,18 @@ typedef enum { SPAVA_SCORE_LOGIT = 0, SPAVA_SCORE_PROB = 1 } spava_score_kind;
  * unknown kind. */
 spava_status spava_plan_set_score_kind(spava_plan* plan, int32_t kind);
 
+/* How spava_attn_prefill (and spava_attn_prefill_noalloc) produce the passing K/V.
+ * enable == 0 (default): the score kernel, then the select + gather kernel.
+ * enable != 0: with the max head reduction over logit scores, scoring, selection and
+ * gather run as one persistent cooperative launch -- score tiles dealt to the SMs in
+ * rounds, each (host, KV head)'s selection started as soon as its last score tile is
+ * stored, its gather shared out over all SMs while later units are still scored.
+ * Plans outside that case run the two kernels either way.  Both give the same scores,
+ * indices and passing K/V (bit for bit); on B200 the two-kernel form is the faster
+ * one at the workloads measured, hence the default.  Host-side only;
+ * SPAVA_ERR_INVALID_ARG for a NULL plan. */
+spava_status spava_plan_set_fused_select(spava_plan* plan, int32_t enable);
+
 /* Bytes of scratch the calls below need (scores, indices, passing K/V, text
  * partials, scheduler counters, error word).  0 if plan is NULL. */
 size_t spava_workspace_bytes(const spava_plan* plan);
@@ -184,7 +196,7 @@ spava_status spava_gather_passing(const spava_plan* plan, const void* k, const v
 
 /*
  * The whole approximate-attention prefill of one layer: scoring -> selection ->
- * gather -> one flash-attention pass per host over
+ * gather (see spava_plan_set_fused_select) -> one flash-attention pass per host over
  * [anchor | passing of hosts < h | own block, causal] (tcgen05/TMEM, bf16 in, fp32
  * accumulation, online softmax) -> text rows as split-KV partials over the host
  * blocks merged through their lse.
@@ -421,7 +433,8 @@ spava_status spava_profile_end(spava_plan* plan);
  * 4 lse merge, 5 attention (dense causal), 6 select + gather (fused, prefill),
  * 7 score-key fill/convert (two-stage), 8 attention stage 1, 9 attention stage 2,
  * 10 probe-row lse (probability scores), 11 passing unpack (sharded prefill),
- * 12 spare text-slot fill (sharded prefill). */
+ * 12 spare text-slot fill (sharded prefill), 13 score + select + gather (one launch,
+ * prefill). */
 const char* spava_kernel_name(int32_t label);
 
 /*

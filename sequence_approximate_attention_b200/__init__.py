@@ -111,6 +111,12 @@ class Plan:
         self.score_kind = kind
         self._refresh_sizes()
 
+    def set_fused_select(self, enable: bool) -> None:
+        """spava_plan_set_fused_select: True scores, selects and gathers in one persistent
+        launch where the plan allows it; False (default) runs the score kernel, then
+        select+gather."""
+        _lib.check(self.lib.spava_plan_set_fused_select(self._h, int(bool(enable))), "spava_plan_set_fused_select")
+
     def _refresh_sizes(self) -> None:
         self.workspace_bytes = int(self.lib.spava_workspace_bytes(self._h))
         self.two_stage_workspace_bytes = int(self.lib.spava_two_stage_workspace_bytes(self._h))

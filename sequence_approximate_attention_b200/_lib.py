@@ -67,6 +67,7 @@ SIGNATURES = {
     "spava_plan_set_debug": (c_int32, [c_void_p, ctypes.c_uint64, c_int32]),
     "spava_plan_set_score_reduce": (c_int32, [c_void_p, c_int32]),
     "spava_plan_set_score_kind": (c_int32, [c_void_p, c_int32]),
+    "spava_plan_set_fused_select": (c_int32, [c_void_p, c_int32]),
     "spava_status_string": (ctypes.c_char_p, [c_int32]),
     "spava_last_error": (ctypes.c_char_p, []),
     "spava_last_launch_count": (c_int32, []),

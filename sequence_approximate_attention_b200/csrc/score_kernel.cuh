@@ -74,10 +74,10 @@ struct ScoreShape {
 // held a different (host, group, chunk).  `items` is the CTA's item range in shared
 // memory.  Written without integer division (q_bufs <= 2): this runs on the MMA
 // thread's critical path once per chunk.
-__device__ __forceinline__ bool score_needs_load(const ScoreParams& p, const int4* items, int li, int c) {
-  int cb = c - p.q_bufs, lb = li;
+__device__ __forceinline__ bool chunk_needs_load(int q_bufs, int n_chunks, const int4* items, int li, int c) {
+  int cb = c - q_bufs, lb = li;
   while (cb < 0) {
-    cb += p.n_chunks;
+    cb += n_chunks;
     --lb;
   }
   if (lb < 0) return true;  // first uses of each buffer
@@ -87,14 +87,211 @@ __device__ __forceinline__ bool score_needs_load(const ScoreParams& p, const int
 }
 
 // The use that comes q_bufs uses after (li, c), as (item, chunk).
-__device__ __forceinline__ void score_next_use(const ScoreParams& p, int li, int c, int* ln, int* cn) {
-  int cc = c + p.q_bufs, l = li;
-  while (cc >= p.n_chunks) {
-    cc -= p.n_chunks;
+__device__ __forceinline__ void chunk_next_use(int q_bufs, int n_chunks, int li, int c, int* ln, int* cn) {
+  int cc = c + q_bufs, l = li;
+  while (cc >= n_chunks) {
+    cc -= n_chunks;
     ++l;
   }
   *ln = l;
   *cn = cc;
+}
+
+// ---------------------------------------------------------------- the scoring pipeline
+// Shared by score_kernel and the fused ssg_kernel: one TMA thread loads 128-key K
+// tiles (a ring of n_stages) and the probe queries; two MMA threads issue the
+// products, issuer X taking the chunk-uses u with u % 2 == X into TMEM accumulator X
+// (columns 256 X ..), so one thread's waits and bookkeeping overlap the other's MMAs
+// on the tensor core; the epilogue drains accumulator u % 2 for use u.
+//
+// Probe-query buffers.  q_bufs == 2 (several chunks per item): buffer X belongs to
+// issuer X (use u reads buffer u % 2) and is reloaded whenever it last held another
+// (host, group, chunk).  q_bufs == 1 (one chunk): the single buffer holds the probe of
+// one (host, group) -- a "generation" of consecutive items -- and is reloaded when the
+// group changes, after every issuer that used it released it (q_empty[X]: one commit
+// per generation the issuer took part in).
+// K stages: released by the issuers that read them (one issuer per item with one
+// chunk, both with more), so k_empty counts 1 or 2 arrivals.
+struct ScorePipe {
+  uint8_t* sQ;
+  uint8_t* sK;
+  int q_bufs, q_buf_bytes, n_stages;
+  uint64_t* k_full;     // [kMaxStages]
+  uint64_t* k_empty;    // [kMaxStages]
+  uint64_t* q_full;     // [2]
+  uint64_t* q_empty;    // [2] per issuer
+  uint64_t* acc_full;   // [2]
+  uint64_t* acc_empty;  // [2], 4 epilogue-warp arrivals
+  uint64_t* drain;      // [2] per issuer
+};
+
+struct ScoreGeom {
+  int probe_r, group, chunk_tokens, n_chunks;
+};
+
+constexpr int kScorePipeStages = 8;  // most K stages any pipeline uses
+constexpr int kScorePipeBarBytes = (2 * kScorePipeStages + 10) * 8;
+
+// Barriers laid out from `bars` (kScorePipeBarBytes); initialised by one thread.
+__device__ __forceinline__ ScorePipe score_pipe_at(uint8_t* sQ, uint8_t* sK, int q_bufs, int q_buf_bytes,
+                                                   int n_stages, uint64_t* bars) {
+  ScorePipe sp;
+  sp.sQ = sQ;
+  sp.sK = sK;
+  sp.q_bufs = q_bufs;
+  sp.q_buf_bytes = q_buf_bytes;
+  sp.n_stages = n_stages;
+  sp.k_full = bars;
+  sp.k_empty = bars + kScorePipeStages;
+  sp.q_full = bars + 2 * kScorePipeStages;
+  sp.q_empty = sp.q_full + 2;
+  sp.acc_full = sp.q_empty + 2;
+  sp.acc_empty = sp.acc_full + 2;
+  sp.drain = sp.acc_empty + 2;
+  return sp;
+}
+
+__device__ __forceinline__ void score_pipe_init(const ScorePipe& sp, int n_chunks) {
+  for (int b = 0; b < sp.n_stages; ++b) {
+    mbar_init(sp.k_full + b, 1);
+    mbar_init(sp.k_empty + b, n_chunks == 1 ? 1 : 2);
+  }
+  for (int b = 0; b < 2; ++b) {
+    mbar_init(sp.q_full + b, 1);
+    mbar_init(sp.q_empty + b, 1);
+    mbar_init(sp.acc_full + b, 1);
+    mbar_init(sp.acc_empty + b, 4);  // one arrival per epilogue warp
+    mbar_init(sp.drain + b, 1);
+  }
+}
+
+__device__ __forceinline__ bool same_group(int4 a, int4 b) { return a.x == b.x && a.y == b.y; }
+
+// TMA producer (one thread): K tile of every item, probe queries when needed.
+template <int D>
+__device__ __forceinline__ void score_produce(const ScorePipe& sp, const ScoreGeom& g, const int4* items,
+                                              int n_local, const CUtensorMap* tmK, const CUtensorMap* tmQp,
+                                              const WaitCtx& wc) {
+  constexpr int kHalves = D / 64, kKTileBytes = kHalves * 128 * 128;
+  const int G = g.group;
+  const uint32_t q_bytes = static_cast<uint32_t>(kHalves * g.chunk_tokens * G * 128);
+  int qloads[2] = {0, 0};       // loads issued into each probe buffer
+  int rel[2] = {0, 0};          // one buffer: releases of each issuer consumed
+  bool part[2] = {false, false};  // one buffer: issuers that used the resident probe
+  int slot = 0, use = 0;        // K stage and how often it was filled before
+  bool ok = true;
+  auto load_q = [&](int b, int4 it, int c) {
+    mbar_arrive_expect_tx(sp.q_full + b, q_bytes);
+    for (int hh = 0; hh < kHalves; ++hh)
+      for (int h = 0; h < G; ++h)
+        tma_load_3d(sp.sQ + b * sp.q_buf_bytes + hh * (g.chunk_tokens * G * 128) + h * (g.chunk_tokens * 128), tmQp,
+                    sp.q_full + b, hh * 64, it.y * G + h, it.w - g.probe_r + c * g.chunk_tokens);
+    ++qloads[b];
+  };
+  for (int li = 0; li < n_local && ok; ++li) {
+    const int4 it = items[li];
+    if (use > 0 && !(ok = mbar_wait(sp.k_empty + slot, (use - 1) & 1, wc, kErrWaitRelease))) break;
+    mbar_arrive_expect_tx(sp.k_full + slot, kKTileBytes);
+    for (int hh = 0; hh < kHalves; ++hh)
+      tma_load_3d(sp.sK + slot * kKTileBytes + hh * 128 * 128, tmK, sp.k_full + slot, hh * 64, it.y, it.z);
+    if (++slot == sp.n_stages) {
+      slot = 0;
+      ++use;
+    }
+    if (sp.q_bufs == 1) {
+      if (li == 0 || !same_group(it, items[li - 1])) {
+        for (int x = 0; x < 2 && ok; ++x)
+          if (part[x]) {
+            ok = mbar_wait(sp.q_empty + x, rel[x] & 1, wc, kErrWaitRelease);
+            ++rel[x];
+          }
+        if (!ok) break;
+        part[0] = part[1] = false;
+        load_q(0, it, 0);
+      }
+      part[li & 1] = true;
+    } else {
+      for (int c = 0; c < g.n_chunks; ++c) {
+        const int b = (li * g.n_chunks + c) & 1;
+        if (!chunk_needs_load(2, g.n_chunks, items, li, c)) continue;
+        if (qloads[b] > 0 && !(ok = mbar_wait(sp.q_empty + b, (qloads[b] - 1) & 1, wc, kErrWaitRelease))) break;
+        load_q(b, it, c);
+      }
+    }
+  }
+  if (!ok) {
+    // Abort: let every copy this thread issued land before the CTA exits.
+    for (int b = 0; b < sp.n_stages; ++b) {
+      const int uses = use + (b < slot ? 1 : 0);
+      if (uses > 0) mbar_wait_drain(sp.k_full + b, (uses - 1) & 1, wc);
+    }
+    for (int b = 0; b < 2; ++b)
+      if (qloads[b] > 0) mbar_wait_drain(sp.q_full + b, (qloads[b] - 1) & 1, wc);
+  }
+}
+
+// MMA issuer X (one thread): S^T = K_tile Qprobe^T for the uses u = X, X + 2, ...
+// into accumulator X.  Never waits on the other issuer.
+template <int D>
+__device__ __forceinline__ void score_issue(const ScorePipe& sp, const ScoreGeom& g, const int4* items, int n_local,
+                                            int X, uint32_t tmem, const WaitCtx& wc) {
+  constexpr int kKTileBytes = (D / 64) * 128 * 128;
+  const int n_uses = n_local * g.n_chunks;
+  const int nc = g.chunk_tokens * g.group;
+  const uint32_t idesc = idesc_bf16_f32(128, nc, 0, 0);
+  const uint32_t qhalf = static_cast<uint32_t>(nc * 128);
+  const uint32_t qa = smem_u32(sp.sQ + (sp.q_bufs == 1 ? 0 : X) * sp.q_buf_bytes);
+  int qwaits = 0;            // two buffers: loads of buffer X waited for
+  int gen = 0, gen_li = 0;   // one buffer: generation (probe load) of item gen_li
+  int my_gen = -1;           // one buffer: the generation this issuer holds
+  bool ok = true, issued_any = false;
+  int li_prev = -1;
+  for (int u = X; u < n_uses && ok; u += 2) {
+    const int li = u / g.n_chunks, c = u - li * g.n_chunks;
+    const int slot = li % sp.n_stages;
+    if (li != li_prev) {
+      if (!(ok = mbar_wait(sp.k_full + slot, (li / sp.n_stages) & 1, wc, kErrWaitLoad))) break;
+      if (sp.q_bufs == 1) {
+        // one buffer: generation k of the probe (its k-th load, phase k of q_full)
+        // starts at the k-th change of group along the items
+        for (; gen_li < li; ++gen_li)
+          if (!same_group(items[gen_li + 1], items[gen_li])) ++gen;
+        if (gen != my_gen) {
+          if (!(ok = mbar_wait(sp.q_full, gen & 1, wc, kErrWaitLoad))) break;
+          my_gen = gen;
+        }
+      }
+      li_prev = li;
+    }
+    if (sp.q_bufs == 2 && chunk_needs_load(2, g.n_chunks, items, li, c)) {
+      if (!(ok = mbar_wait(sp.q_full + X, qwaits & 1, wc, kErrWaitLoad))) break;
+      ++qwaits;
+    }
+    if (u >= 2 && !(ok = mbar_wait(sp.acc_empty + X, ((u >> 1) - 1) & 1, wc, kErrWaitMma))) break;
+    tc_fence_after();
+    const uint32_t ka = smem_u32(sp.sK + slot * kKTileBytes);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+      const uint32_t qoff = (kk >> 2) * qhalf + (kk & 3) * 32;
+      mma_ss(tmem + X * 256, sdesc_sw128(ka + koff, 16, 1024), sdesc_sw128(qa + qoff, 16, 1024), idesc,
+             kk > 0 ? 1u : 0u);
+    }
+    mma_commit(sp.acc_full + X);
+    issued_any = true;
+    const int un = u + 2;
+    const int ln = un < n_uses ? un / g.n_chunks : -1;
+    if (sp.q_bufs == 1) {
+      if (ln < 0 || !same_group(items[ln], items[li])) mma_commit(sp.q_empty + X);
+    } else if (ln >= 0 && chunk_needs_load(2, g.n_chunks, items, ln, un - ln * g.n_chunks)) {
+      mma_commit(sp.q_empty + X);
+    }
+    if (ln != li) mma_commit(sp.k_empty + slot);  // this issuer's last use of the K tile
+  }
+  if (issued_any) {
+    mma_commit(sp.drain + X);
+    mbar_wait_drain(sp.drain + X, 0, wc);
+  }
 }
 
 template <int D>
@@ -106,33 +303,17 @@ __global__ void __launch_bounds__(256, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int n_stages = p.k_stages;
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + p.q_bufs * p.q_buf_bytes;   // q_buf_bytes is a multiple of 1024
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sK + n_stages * S::kKTileBytes);
-  uint64_t* k_full = bars + 0;                   // [kMaxStages]
-  uint64_t* k_empty = k_full + S::kMaxStages;    // [kMaxStages]
-  uint64_t* q_full = k_empty + S::kMaxStages;    // [2]
-  uint64_t* q_empty = q_full + 2;                // [2]
-  uint64_t* acc_full = q_empty + 2;              // [2]
-  uint64_t* acc_empty = acc_full + 2;            // [2]
-  uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  int4* s_items = reinterpret_cast<int4*>(reinterpret_cast<uint8_t*>(bars) + S::kBarBytes);
+  uint8_t* sK = smem + p.q_bufs * p.q_buf_bytes;  // q_buf_bytes is a multiple of 1024
+  uint8_t* bar_base = sK + n_stages * S::kKTileBytes;
+  const ScorePipe sp = score_pipe_at(smem, sK, p.q_bufs, p.q_buf_bytes, n_stages, reinterpret_cast<uint64_t*>(bar_base));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_base + kScorePipeBarBytes);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int4* s_items = reinterpret_cast<int4*>(bar_base + S::kBarBytes);
+  const ScoreGeom geom{p.probe_r, p.group, p.chunk_tokens, p.n_chunks};
 
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
-    for (int b = 0; b < n_stages; ++b) {
-      mbar_init(k_full + b, 1);
-      mbar_init(k_empty + b, 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(q_full + b, 1);
-      mbar_init(q_empty + b, 1);
-      mbar_init(acc_full + b, 1);
-      mbar_init(acc_empty + b, 4);  // one arrival per epilogue warp
-    }
-    mbar_init(drain, 1);
+    score_pipe_init(sp, p.n_chunks);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -153,96 +334,10 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (lane 0)
-    if (lane == 0) {
-      int qloads[2] = {0, 0};
-      int slot = 0, use = 0;  // K stage and how often it was filled before (no division)
-      bool ok = true;
-      for (int li = 0; li < n_local && ok; ++li) {
-        const int4 it = s_items[li];
-        if (use > 0 && !(ok = mbar_wait(k_empty + slot, (use - 1) & 1, wc, kErrWaitRelease))) break;
-        mbar_arrive_expect_tx(k_full + slot, S::kKTileBytes);
-        for (int hh = 0; hh < S::kHalves; ++hh)
-          tma_load_3d(sK + slot * S::kKTileBytes + hh * 128 * 128, &tmK, k_full + slot, hh * 64, it.y, it.z);
-        if (++slot == n_stages) {
-          slot = 0;
-          ++use;
-        }
-        for (int c = 0; c < p.n_chunks; ++c) {
-          const int u = li * p.n_chunks + c, b = u & (p.q_bufs - 1);
-          if (!score_needs_load(p, s_items, li, c)) continue;
-          if (qloads[b] > 0 && !(ok = mbar_wait(q_empty + b, (qloads[b] - 1) & 1, wc, kErrWaitRelease))) break;
-          mbar_arrive_expect_tx(q_full + b, static_cast<uint32_t>(S::kHalves * p.chunk_tokens * G * 128));
-          for (int hh = 0; hh < S::kHalves; ++hh)
-            for (int h = 0; h < G; ++h)
-              tma_load_3d(sQ + b * p.q_buf_bytes + hh * (p.chunk_tokens * G * 128) + h * (p.chunk_tokens * 128), &tmQp,
-                          q_full + b, hh * 64, it.y * G + h, it.w - p.probe_r + c * p.chunk_tokens);
-          ++qloads[b];
-        }
-      }
-      if (!ok) {
-        // Abort: let every copy this thread issued land before the CTA exits.
-        for (int b = 0; b < n_stages; ++b) {
-          const int uses = use + (b < slot ? 1 : 0);  // loads issued into stage b
-          if (uses > 0) mbar_wait_drain(k_full + b, (uses - 1) & 1, wc);
-        }
-        for (int b = 0; b < 2; ++b)
-          if (qloads[b] > 0) mbar_wait_drain(q_full + b, (qloads[b] - 1) & 1, wc);
-      }
-    }
+    if (lane == 0) score_produce<D>(sp, geom, s_items, n_local, &tmK, &tmQp, wc);
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (lane 0)
-    // One thread issues every MMA (tcgen05.mma returns once the tensor core has taken
-    // the instruction), with no warp-wide votes between them.
-    if (lane == 0) {
-      int qloads[2] = {0, 0};
-      bool ok = true, issued_any = false;
-      int slot = 0, kphase = 0;
-      for (int li = 0; li < n_local && ok; ++li) {
-        if (!(ok = mbar_wait(k_full + slot, kphase, wc, kErrWaitLoad))) break;
-        for (int c = 0; c < p.n_chunks; ++c) {
-          const int u = li * p.n_chunks + c;
-          const int qb = u & (p.q_bufs - 1);  // probe-query buffer (q_bufs is 1 or 2)
-          const int ab = u & 1;               // TMEM accumulator
-          if (score_needs_load(p, s_items, li, c)) {
-            ok = mbar_wait(q_full + qb, qloads[qb] & 1, wc, kErrWaitLoad);
-            ++qloads[qb];
-            if (!ok) break;
-          }
-          if (u >= 2 && !(ok = mbar_wait(acc_empty + ab, ((u >> 1) - 1) & 1, wc, kErrWaitMma))) break;
-          tc_fence_after();
-          // All Rc G columns: with (head, token) order a short last chunk's probe rows
-          // are not a prefix; the epilogue masks the rest.
-          const int nc = p.chunk_tokens * G;
-          const uint32_t idesc = idesc_bf16_f32(128, nc, 0, 0);
-          const uint32_t ka = smem_u32(sK + slot * S::kKTileBytes);
-          const uint32_t qa = smem_u32(sQ + qb * p.q_buf_bytes);
-          const uint32_t qhalf = static_cast<uint32_t>(p.chunk_tokens * G * 128);
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            const uint32_t qoff = (kk >> 2) * qhalf + (kk & 3) * 32;
-            mma_ss(tmem + ab * 256, sdesc_sw128(ka + koff, 16, 1024), sdesc_sw128(qa + qoff, 16, 1024), idesc,
-                   kk > 0 ? 1u : 0u);
-          }
-          mma_commit(acc_full + ab);
-          int ln, cn;
-          score_next_use(p, li, c, &ln, &cn);
-          if (ln < n_local && score_needs_load(p, s_items, ln, cn)) mma_commit(q_empty + qb);
-          issued_any = true;
-        }
-        if (!ok) break;
-        mma_commit(k_empty + slot);
-        if (++slot == n_stages) {
-          slot = 0;
-          kphase ^= 1;
-        }
-      }
-      if (issued_any) {
-        mma_commit(drain);
-        mbar_wait_drain(drain, 0, wc);
-      }
-    }
+  } else if (warp == 1 || warp == 3) {
+    if (lane == 0) score_issue<D>(sp, geom, s_items, n_local, warp == 1 ? 0 : 1, tmem, wc);
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue: one key per thread
@@ -265,7 +360,7 @@ __global__ void __launch_bounds__(256, 1)
       }
       for (int c = 0; c < p.n_chunks; ++c) {
         const int u = li * p.n_chunks + c, b = u & 1;
-        ok = __all_sync(FULL, mbar_wait(acc_full + b, (u >> 1) & 1, wc, kErrWaitMma));
+        ok = __all_sync(FULL, mbar_wait(sp.acc_full + b, (u >> 1) & 1, wc, kErrWaitMma));
         if (!ok) break;
         tc_fence_after();
         const int row0 = e - p.probe_r + c * Rc;         // first probe row of the chunk
@@ -331,7 +426,7 @@ __global__ void __launch_bounds__(256, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty + b);
+        if (lane == 0) mbar_arrive(sp.acc_empty + b);
       }
       if (!ok) break;
       const float out_scale = prob ? 1.0f : p.scale;  // probabilities carry the scale already

@@ -26,6 +26,7 @@
 #include "common.cuh"
 #include "proj_kernel.cuh"
 #include "score_kernel.cuh"
+#include "ssg_kernel.cuh"
 #include "select_gather.cuh"
 
 using spava::AttnItem;
@@ -120,6 +121,7 @@ struct spava_plan {
   int rc = 0, n_chunks = 0;
   int score_reduce = SPAVA_SCORE_MAX;  // spava_plan_set_score_reduce
   int score_kind = SPAVA_SCORE_LOGIT;  // spava_plan_set_score_kind
+  int fused_select = 0;                // spava_plan_set_fused_select
   // device table (owned)
   void* dtab = nullptr;
   int* d_off = nullptr;
@@ -137,6 +139,11 @@ struct spava_plan {
   int n_score_pre = 0;
   int4* d_score_all = nullptr;  // all hosts
   int n_score_all = 0;
+  // fused score/select/gather: hosts 0..H-2's score tiles dealt to ssg_grid CTAs in
+  // rounds; CTA b takes d_ssg_items[d_ssg_first[b] .. d_ssg_first[b+1])
+  int4* d_ssg_items = nullptr;
+  int* d_ssg_first = nullptr;
+  int ssg_grid = 0, ssg_max_local = 0;
   // sharded prefill (spava_plan_set_shard): this rank's work lists in their own
   // device table; the exchange buffers' slots per rank
   int shard_rank = 0, shard_world = 0;  // world 0: not sharded
@@ -158,7 +165,7 @@ struct spava_plan {
   AttnItem* d_items_shard_pre = nullptr;  // one-pass form (SPAVA_SHARD_ATTEND)
   int n_items_shard_pre = 0;
   // workspace layout
-  size_t ws_err = 0, ws_scores = 0, ws_idx = 0, ws_kp = 0, ws_vp = 0, ws_opart = 0, ws_lpart = 0, ws_total = 0;
+  size_t ws_err = 0, ws_sync = 0, ws_scores = 0, ws_idx = 0, ws_kp = 0, ws_vp = 0, ws_opart = 0, ws_lpart = 0, ws_total = 0;
   size_t ws_row_o = 0, ws_row_lse = 0, ws_qkeys = 0, ws_total_two_stage = 0;  // two-stage flow only
   size_t ws_probe_lse = 0;  // probability scores: [hq][N] lse (probe rows only)
   size_t ws_xk = 0, ws_xv = 0, ws_to = 0, ws_tl = 0, ws_total_shard = 0;  // sharded prefill
@@ -178,7 +185,8 @@ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 enum KernelLabel {
   kLabScore = 0, kLabSelect = 1, kLabGather = 2, kLabAttn = 3, kLabMerge = 4, kLabDense = 5, kLabSelectGather = 6,
-  kLabFill = 7, kLabAttnLocal = 8, kLabAttnRemote = 9, kLabProbeLse = 10, kLabUnpack = 11, kLabTextFill = 12
+  kLabFill = 7, kLabAttnLocal = 8, kLabAttnRemote = 9, kLabProbeLse = 10, kLabUnpack = 11, kLabTextFill = 12,
+  kLabScoreSelectGather = 13
 };
 
 void mark(const spava_plan* p, int label, cudaStream_t st) {
@@ -394,6 +402,33 @@ std::vector<int4> build_score_items(const spava_plan& p, int h_end, const HostMa
   return v;
 }
 
+// Score tiles `v` (unit order) dealt to `grid` CTAs in rounds, for the fused
+// score/select/gather launch: CTA b takes n / grid tiles (+-1) in `rounds` near-equal
+// chunks, and round r hands every CTA, in CTA order, its r-th chunk from the next
+// stretch of the list.  A unit is then complete once the round holding its last tile
+// is scored everywhere, so units complete round after round instead of all at the
+// end.  Rounds: about one per ten tiles of a CTA (a new chunk usually reloads the
+// probe queries), at most 8.
+void deal_rounds(const std::vector<int4>& v, int grid, std::vector<int4>* out, std::vector<int>* first) {
+  const int n = static_cast<int>(v.size());
+  const int per = ceil_div(n, grid);
+  const int rounds = std::max(1, std::min(8, (per + 5) / 10));
+  std::vector<int> tot(grid);
+  first->assign(grid + 1, 0);
+  for (int b = 0; b < grid; ++b) {
+    tot[b] = static_cast<int>(static_cast<long long>(n) * (b + 1) / grid - static_cast<long long>(n) * b / grid);
+    (*first)[b + 1] = (*first)[b] + tot[b];
+  }
+  out->assign(v.size(), make_int4(0, 0, 0, 0));
+  std::vector<int> placed(grid, 0);
+  int pos = 0;
+  for (int r = 0; r < rounds; ++r)
+    for (int b = 0; b < grid; ++b) {
+      const int sz = tot[b] * (r + 1) / rounds - tot[b] * r / rounds;
+      for (int k = 0; k < sz; ++k) (*out)[(*first)[b] + placed[b]++] = v[pos++];
+    }
+}
+
 template <class K>
 spava_status ensure_smem(K kernel, int bytes) {
   SPAVA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
@@ -417,6 +452,8 @@ void layout_workspace(spava_plan* p) {
   size_t o = 0;
   p->ws_err = o;
   o += 256;
+  p->ws_sync = o;  // fused score/select/gather: unit counters and ready flags
+  o = align_up(o + 2 * hm1 * rows * 4, 256);
   p->ws_scores = o;
   o = align_up(o + rows * n_visual * 4, 256);
   p->ws_idx = o;
@@ -561,6 +598,104 @@ spava_status launch_select(const spava_plan* p, const float* scores, int32_t* id
   return SPAVA_OK;
 }
 
+// Grid of the fused score/select/gather launch (ssg_kernel.cuh) for this plan, or 0
+// when the plan is outside what that kernel covers (another head reduction or score
+// kind, the fused path switched off, more score tiles per CTA than it caches, or a
+// grid that cannot be resident at once); the prefill then takes the score kernel and
+// the select+gather kernel.  Sets *smem_out and *task_rows_out.
+template <int D>
+int ssg_grid(const spava_plan* p, int* smem_out, int* k_stages_out, int* task_rows_out) {
+  using S = spava::SsgShape<D>;
+  if (!p->fused_select || p->score_reduce != SPAVA_SCORE_MAX || p->score_kind != SPAVA_SCORE_LOGIT) return 0;
+  if (p->H < 2 || p->P == 0 || p->n_score_pre == 0) return 0;
+  const int grid = p->ssg_grid;
+  if (grid <= 0 || p->ssg_max_local > S::kMaxLocalItems) return 0;
+  const int G = p->hq / p->hkv;
+  const int q_bufs = p->n_chunks == 1 ? 1 : 2, q_buf_bytes = (D / 64) * p->rc * G * 128;
+  const int k_stages =
+      std::min<int>(S::kMaxStages, (S::kSmemMax - S::smem_bytes(q_bufs, q_buf_bytes, 0)) / S::kKTileBytes);
+  if (k_stages < 2) return 0;
+  const int smem = S::smem_bytes(q_bufs, q_buf_bytes, k_stages);
+  if (ensure_smem(spava::ssg_kernel<D>, S::kSmemMax) != SPAVA_OK) return 0;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, spava::ssg_kernel<D>, S::kThreads, smem) != cudaSuccess)
+    return 0;
+  if (per_sm < 1 || grid > per_sm * p->num_sms) return 0;
+  // gather tasks: at most kMaxOwnTasks per CTA
+  const int n_units = (p->H - 1) * p->hkv;
+  int task_rows = 128;
+  while (static_cast<long long>(n_units) * ceil_div(p->P, task_rows) > static_cast<long long>(S::kMaxOwnTasks) * grid)
+    task_rows *= 2;
+  *smem_out = smem;
+  *k_stages_out = k_stages;
+  *task_rows_out = task_rows;
+  return grid;
+}
+
+// Scores, selection and passing K/V of hosts 0..H-2 in one cooperative launch.  The
+// unit counters and ready flags (workspace, ws_sync) must be zero: begin_call clears
+// them.  `grid`, `smem`, `k_stages` and `task_rows` come from ssg_grid.
+template <int D>
+spava_status launch_ssg(const spava_plan* p, int grid, int smem, int k_stages, int task_rows, const void* q,
+                        const void* k, const void* v, float* scores, int32_t* idx, void* kp, void* vp, void* ws,
+                        cudaStream_t st) {
+  using S = spava::SsgShape<D>;
+  CUtensorMap tmK, tmQp;
+  spava_status s;
+  if ((s = make_map(&tmK, k, D, p->hkv, p->N + p->T, 1, 128)) != SPAVA_OK) return s;
+  if ((s = make_map(&tmQp, q, D, p->hq, p->N + p->T, 1, p->rc)) != SPAVA_OK) return s;
+  const int G = p->hq / p->hkv;
+  const int n_units = (p->H - 1) * p->hkv;
+  const size_t cpr = static_cast<size_t>(D) * 2 / 16;
+  spava::SsgParams sp{};
+  sp.items = p->d_ssg_items;
+  sp.cta_first = p->d_ssg_first;
+  sp.probe_r = p->R;
+  sp.group = G;
+  sp.chunk_tokens = p->rc;
+  sp.n_chunks = p->n_chunks;
+  sp.n_visual = p->N;
+  sp.scale = p->scale;
+  sp.scores = scores;
+  sp.q_bufs = p->n_chunks == 1 ? 1 : 2;
+  sp.q_buf_bytes = (D / 64) * p->rc * G * 128;
+  sp.k_stages = k_stages;
+  sp.off = p->d_off;
+  sp.hkv = p->hkv;
+  sp.anchor = p->A;
+  sp.passing = p->P;
+  sp.unit_cnt = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + p->ws_sync);
+  sp.unit_ready = sp.unit_cnt + n_units;
+  sp.idx = idx;
+  sp.k = static_cast<const uint4*>(k);
+  sp.v = static_cast<const uint4*>(v);
+  sp.kp = static_cast<uint4*>(kp);
+  sp.vp = static_cast<uint4*>(vp);
+  sp.chunks_per_row = static_cast<int>(cpr);
+  sp.dst_h = static_cast<size_t>(p->P) * cpr;
+  sp.dst_g = static_cast<size_t>(p->H - 1) * sp.dst_h;
+  sp.task_rows = task_rows;
+  sp.tasks_per_unit = ceil_div(p->P, task_rows);
+  sp.n_tasks = n_units * sp.tasks_per_unit;
+  sp.err_word = err_word(p, ws);
+  sp.wait_limit_ns = p->wait_limit_ns;
+  sp.stall_producer = p->stall_producer;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(S::kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  mark(p, kLabScoreSelectGather, st);
+  SPAVA_CUDA(cudaLaunchKernelEx(&cfg, spava::ssg_kernel<D>, tmK, tmQp, sp));
+  ++g_last_launches;
+  return SPAVA_OK;
+}
+
 spava_status launch_gather(const spava_plan* p, const void* k, const void* v, const int32_t* idx, void* kp, void* vp,
                            cudaStream_t st) {
   if (p->H < 2 || p->P == 0) return SPAVA_OK;
@@ -686,7 +821,8 @@ spava_status begin_call(const spava_plan* p, void* ws, cudaStream_t st, bool cle
   int dev = -1;
   SPAVA_CUDA(cudaGetDevice(&dev));
   if (dev != p->device) return fail(SPAVA_ERR_INVALID_ARG, "current device %d differs from the plan's device %d", dev, p->device);
-  if (clear_error) SPAVA_CUDA(cudaMemsetAsync(err_word(p, ws), 0, 256, st));
+  // the error word and the fused launch's counters, which must start at zero
+  if (clear_error) SPAVA_CUDA(cudaMemsetAsync(err_word(p, ws), 0, p->ws_scores - p->ws_err, st));
   return SPAVA_OK;
 }
 
@@ -825,6 +961,13 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   p->n_items_probe = static_cast<int>(probe.size());
   p->n_score_pre = static_cast<int>(sc_pre.size());
   p->n_score_all = static_cast<int>(sc_all.size());
+  std::vector<int4> ssg_items;
+  std::vector<int> ssg_first;
+  p->ssg_grid = std::min(p->n_score_pre, p->num_sms);
+  if (p->ssg_grid > 0) {
+    deal_rounds(sc_pre, p->ssg_grid, &ssg_items, &ssg_first);
+    for (int b = 0; b < p->ssg_grid; ++b) p->ssg_max_local = std::max(p->ssg_max_local, ssg_first[b + 1] - ssg_first[b]);
+  }
   // One device table, each array 256-byte aligned.
   TablePacker tab;
   const size_t o_off = tab.put(off.data(), off.size() * 4);
@@ -835,6 +978,8 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   const size_t o_local = tab.put(local.data(), local.size() * sizeof(AttnItem));
   const size_t o_remote = tab.put(remote.data(), remote.size() * sizeof(AttnItem));
   const size_t o_probe = tab.put(probe.data(), probe.size() * sizeof(AttnItem));
+  const size_t o_ssg_items = tab.put(ssg_items.data(), ssg_items.size() * sizeof(int4));
+  const size_t o_ssg_first = tab.put(ssg_first.data(), ssg_first.size() * 4);
   spava_status ust = upload_table(tab.host, &p->dtab);
   if (ust != SPAVA_OK) return bail(ust);
   uint8_t* base = static_cast<uint8_t*>(p->dtab);
@@ -846,6 +991,8 @@ spava_status spava_plan_create(spava_plan** out, int32_t n_visual, int32_t n_tex
   p->d_items_local = reinterpret_cast<AttnItem*>(base + o_local);
   p->d_items_remote = reinterpret_cast<AttnItem*>(base + o_remote);
   p->d_items_probe = reinterpret_cast<AttnItem*>(base + o_probe);
+  p->d_ssg_items = reinterpret_cast<int4*>(base + o_ssg_items);
+  p->d_ssg_first = reinterpret_cast<int*>(base + o_ssg_first);
   *out = p;
   return ok();
 }
@@ -889,6 +1036,12 @@ spava_status spava_plan_set_score_kind(spava_plan* p, int32_t kind) {
     return fail(SPAVA_ERR_INVALID_ARG, "unknown score kind %d", kind);
   p->score_kind = kind;
   layout_workspace(p);  // probability scores keep the probe rows' lse in the workspace
+  return ok();
+}
+
+spava_status spava_plan_set_fused_select(spava_plan* p, int32_t enable) {
+  if (!p) return fail(SPAVA_ERR_INVALID_ARG, "plan is NULL");
+  p->fused_select = enable ? 1 : 0;
   return ok();
 }
 
@@ -951,11 +1104,20 @@ spava_status spava_attn_prefill(const spava_plan* p, const void* q, const void* 
   void* kp = w + p->ws_kp;
   void* vp = w + p->ws_vp;
   if (p->H >= 2 && p->P > 0) {
-    if ((s = launch_probe_lse(p, q, k, v, ws, st)) != SPAVA_OK) return s;
-    s = p->d == 128 ? launch_score<128>(p, q, k, scores, p->d_score_pre, p->n_score_pre, ws, st)
-                    : launch_score<64>(p, q, k, scores, p->d_score_pre, p->n_score_pre, ws, st);
-    if (s != SPAVA_OK) return s;
-    if ((s = launch_select(p, scores, idx, st, k, v, PassDest{kp, vp, false})) != SPAVA_OK) return s;
+    int smem = 0, k_stages = 0, task_rows = 0;
+    const int grid = p->d == 128 ? ssg_grid<128>(p, &smem, &k_stages, &task_rows)
+                                 : ssg_grid<64>(p, &smem, &k_stages, &task_rows);
+    if (grid > 0) {
+      s = p->d == 128 ? launch_ssg<128>(p, grid, smem, k_stages, task_rows, q, k, v, scores, idx, kp, vp, ws, st)
+                      : launch_ssg<64>(p, grid, smem, k_stages, task_rows, q, k, v, scores, idx, kp, vp, ws, st);
+      if (s != SPAVA_OK) return s;
+    } else {
+      if ((s = launch_probe_lse(p, q, k, v, ws, st)) != SPAVA_OK) return s;
+      s = p->d == 128 ? launch_score<128>(p, q, k, scores, p->d_score_pre, p->n_score_pre, ws, st)
+                      : launch_score<64>(p, q, k, scores, p->d_score_pre, p->n_score_pre, ws, st);
+      if (s != SPAVA_OK) return s;
+      if ((s = launch_select(p, scores, idx, st, k, v, PassDest{kp, vp, false})) != SPAVA_OK) return s;
+    }
   }
   s = p->d == 128 ? launch_attn<128>(p, p->d_items_pre, p->n_items_pre, q, k, v, kp, vp, o, lse, ws, st)
                   : launch_attn<64>(p, p->d_items_pre, p->n_items_pre, q, k, v, kp, vp, o, lse, ws, st);
@@ -1406,6 +1568,7 @@ const char* spava_kernel_name(int32_t label) {
     case kLabProbeLse: return "probe_lse";
     case kLabUnpack: return "unpack_passing";
     case kLabTextFill: return "text_slot_fill";
+    case kLabScoreSelectGather: return "score_select_gather";
   }
   return "unknown";
 }
