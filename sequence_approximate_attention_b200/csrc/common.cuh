@@ -18,6 +18,8 @@ enum : uint32_t {
   kErrWaitSoftmax = 1u << 2,  // the MMA warp waited too long for softmax output
   kErrWaitRelease = 1u << 3,  // the load warp waited too long for a free buffer
   kErrWaitDrain = 1u << 4,    // an abort could not drain copies in flight
+  kErrWaitUnit = 1u << 5,     // a wait on another CTA's or warp's progress in the fused launch ran out
+  kErrBadIndex = 1u << 6,     // a selection or gather index fell outside its range (the access was skipped)
 };
 
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s

@@ -35,13 +35,9 @@
 
 #include "common.cuh"
 #include "score_kernel.cuh"
+#include "topp_select.cuh"
 
 namespace spava {
-
-enum : uint32_t {
-  kErrWaitUnit = 1u << 5,  // a wait on another CTA's or warp's progress in the fused launch ran out
-  kErrBadIndex = 1u << 6,  // a selection or gather index fell outside its range (the access was skipped)
-};
 
 struct SsgParams {
   // scoring
@@ -78,9 +74,7 @@ struct SsgParams {
 
 // Shared state of the worker group, the publisher and the hand-off ring.
 struct SsgCtl {
-  uint32_t hist[2048];
-  uint32_t scan[40];
-  uint32_t sel_prefix, sel_k;
+  ToppShared sel;  // the worker group's selection scratch
   int ring[32];    // units this CTA completed, + 1 (0 = empty slot)
   int ring_tail;   // slots the publisher filled
   int stored;      // epilogue-warp arrivals: 4 per score tile stored
@@ -118,6 +112,9 @@ __device__ __forceinline__ void worker_bar() {
   __syncwarp();
   asm volatile("barrier.sync %0, %1;" ::"n"(kSsgBar), "n"(256) : "memory");
 }
+struct WorkerBar {
+  __device__ __forceinline__ void operator()() const { worker_bar(); }
+};
 
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   int v;
@@ -136,212 +133,7 @@ __device__ __forceinline__ void red_release_cta_shared_add(int* p, int v) {
   asm volatile("red.release.cta.shared::cta.add.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
 }
 
-// Exclusive prefix sum over the 256 worker threads (wt = worker thread index).
-__device__ __forceinline__ uint32_t worker_exclusive_scan(uint32_t v, uint32_t* scratch, int wt) {
-  const int lane = wt & 31, w = wt >> 5;
-  uint32_t incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) scratch[w] = incl;
-  worker_bar();
-  if (w == 0) {
-    const uint32_t x = lane < 8 ? scratch[lane] : 0u;
-    uint32_t xi = x;
-#pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, xi, o);
-      if (lane >= o) xi += y;
-    }
-    if (lane < 8) scratch[8 + lane] = xi - x;  // exclusive warp offsets
-  }
-  worker_bar();
-  const uint32_t res = scratch[8 + w] + incl - v;
-  worker_bar();
-  return res;
-}
-
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-
-// Exclusive prefix of per-(row, warp) counts in index order over one block of 32
-// rows of 256 keys: lane i of warp w holds the count of row i; returns, in lane i, the
-// number of counted keys before (row i, warp w), and the block's total in *total.
-// grid: 256 words of shared memory.
-__device__ __forceinline__ uint32_t row_warp_scan(uint32_t cnt_of_lane_row, uint32_t* grid, uint32_t* scratch,
-                                                  int wt, uint32_t* total) {
-  const int lane = wt & 31, w = wt >> 5;
-  grid[lane * 8 + w] = cnt_of_lane_row;  // (row, warp) in index order
-  worker_bar();
-  const uint32_t v = grid[wt];
-  const uint32_t ex = worker_exclusive_scan(v, scratch, wt);
-  grid[wt] = ex;
-  if (wt == 255) scratch[20] = ex + v;
-  worker_bar();
-  const uint32_t r = grid[lane * 8 + w];
-  *total = scratch[20];
-  worker_bar();
-  return r;
-}
-
-// Top-P of the n candidate scores s[0..n) (token lo + i) by the worker group.
-// Thread wt owns keys i * 256 + wt (rows i of 256 keys, read coalesced); with kPer > 0
-// (n <= 256 kPer, kPer <= 32) they stay in registers, else every pass reads them again
-// from L2.  Radix select of the P-th largest ordered key T: the bits every key shares
-// (from the block's min and max) are known at once, the rest is resolved in digits of
-// up to 11 bits, most significant first.  Then a stable compaction in index order
-// (row, warp, lane): keys > T, and the keys == T of lowest index up to P in all,
-// written ascending to out[0..P).
-template <int kPer>
-__device__ __forceinline__ void ssg_select(const float* s, int n, int lo, int passing, int32_t* out, SsgCtl* c,
-                                           int wt, unsigned int* err_word) {
-  constexpr int NT = 256;
-  constexpr uint32_t FULL = 0xffffffffu;
-  const int lane = wt & 31, w = wt >> 5;
-  const int rows = (n + NT - 1) / NT;
-  constexpr int kRegs = kPer > 0 ? kPer : 1;
-  uint32_t u[kRegs];
-  if (kPer > 0) {
-#pragma unroll
-    for (int i = 0; i < kRegs; ++i) u[i] = i * NT + wt < n ? ordered_key(__ldcg(s + i * NT + wt)) : 0u;
-  }
-  auto key = [&](int i) -> uint32_t { return kPer > 0 ? u[i] : ordered_key(__ldcg(s + i * NT + wt)); };
-  const int n_loop = kPer > 0 ? kRegs : rows;
-
-  // min and max key: the common leading bits of every key
-  uint32_t kmin = 0xffffffffu, kmax = 0u;
-#pragma unroll
-  for (int i = 0; i < n_loop; ++i) {
-    if (i * NT + wt < n) {
-      const uint32_t x = key(i);
-      kmin = min(kmin, x);
-      kmax = max(kmax, x);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(FULL, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(FULL, kmax, o));
-  }
-  if (lane == 0) {
-    c->scan[24 + w] = kmin;
-    c->scan[32 + w] = kmax;
-  }
-  worker_bar();
-  kmin = c->scan[24];
-  kmax = c->scan[32];
-  for (int x = 1; x < 8; ++x) {
-    kmin = min(kmin, c->scan[24 + x]);
-    kmax = max(kmax, c->scan[32 + x]);
-  }
-  worker_bar();
-  const int cp = kmin == kmax ? 32 : __clz(kmin ^ kmax);  // leading bits all keys share
-  uint32_t pmask = cp == 32 ? 0xffffffffu : ~(0xffffffffu >> cp);
-  uint32_t prefix = kmax & pmask, k = static_cast<uint32_t>(passing);
-  int shift = 32 - cp;
-#pragma unroll 1
-  while (shift > 0) {
-    const int wd = min(11, shift);
-    shift -= wd;
-    const int nb = 1 << wd;  // bins of this digit
-    const uint32_t dmask = static_cast<uint32_t>(nb - 1);
-    for (int b = wt; b < nb; b += NT) c->hist[b] = 0u;
-    worker_bar();
-#pragma unroll
-    for (int i = 0; i < n_loop; ++i) {
-      if (i * NT + wt < n) {
-        const uint32_t x = key(i);
-        if ((x & pmask) == prefix) atomicAdd(&c->hist[(x >> shift) & dmask], 1u);
-      }
-    }
-    worker_bar();
-    // thread wt owns bins top .. top-bpt+1 (descending order of keys)
-    const int bpt = nb >= NT ? nb / NT : 1;
-    const int top = nb - 1 - wt * bpt;
-    uint32_t sum = 0u;
-    for (int t = 0; t < bpt && top - t >= 0; ++t) sum += c->hist[top - t];
-    const uint32_t excl = worker_exclusive_scan(sum, c->scan, wt);
-    if (excl < k && k <= excl + sum) {
-      uint32_t acc = excl;
-      for (int t = 0; t < bpt; ++t) {
-        const uint32_t cb = c->hist[top - t];
-        if (acc + cb >= k) {
-          c->sel_prefix = prefix | (static_cast<uint32_t>(top - t) << shift);
-          c->sel_k = k - acc;
-          break;
-        }
-        acc += cb;
-      }
-    }
-    worker_bar();
-    prefix = c->sel_prefix;
-    k = c->sel_k;
-    pmask |= dmask << shift;
-  }
-  const uint32_t T = prefix;   // key of the P-th largest score
-  const uint32_t take_eq = k;  // keys equal to T that are taken (lowest index first)
-
-  // compaction over blocks of 32 rows, in index order (row, warp, lane); with the keys
-  // in registers there is one block and the row loops unroll (static register indices)
-  uint32_t* grid = c->hist;  // 256 words
-  const uint32_t below = (1u << lane) - 1u;
-  constexpr int kRowsPerBlock = kPer > 0 ? kRegs : 32;
-  uint32_t eq_base = 0u, win_base = 0u;
-#pragma unroll 1
-  for (int r0 = 0; r0 < rows; r0 += 32) {
-    const int rb = min(32, rows - r0);
-    uint32_t eq_cnt = 0u;
-#pragma unroll
-    for (int i = 0; i < kRowsPerBlock; ++i) {
-      if (i < rb) {
-        const int ii = r0 + i;
-        const bool e = ii * NT + wt < n && key(kPer > 0 ? i : ii) == T;
-        const uint32_t m = __popc(__ballot_sync(FULL, e));
-        if (lane == i) eq_cnt = m;
-      }
-    }
-    uint32_t tot_eq;
-    const uint32_t eq_before = row_warp_scan(eq_cnt, grid, c->scan, wt, &tot_eq);  // lane i: row r0 + i
-    uint32_t win_cnt = 0u;
-#pragma unroll
-    for (int i = 0; i < kRowsPerBlock; ++i) {
-      if (i < rb) {
-        const int ii = r0 + i;
-        const bool valid = ii * NT + wt < n;
-        const uint32_t x = valid ? key(kPer > 0 ? i : ii) : 0u;
-        const uint32_t eb = __ballot_sync(FULL, valid && x == T);
-        const uint32_t rank = eq_base + __shfl_sync(FULL, eq_before, i) + __popc(eb & below);
-        const bool win = valid && (x > T || (x == T && rank < take_eq));
-        const uint32_t m = __popc(__ballot_sync(FULL, win));
-        if (lane == i) win_cnt = m;
-      }
-    }
-    uint32_t tot_win;
-    const uint32_t win_before = row_warp_scan(win_cnt, grid, c->scan, wt, &tot_win);
-#pragma unroll
-    for (int i = 0; i < kRowsPerBlock; ++i) {
-      if (i < rb) {
-        const int ii = r0 + i;
-        const bool valid = ii * NT + wt < n;
-        const uint32_t x = valid ? key(kPer > 0 ? i : ii) : 0u;
-        const uint32_t eb = __ballot_sync(FULL, valid && x == T);
-        const uint32_t rank = eq_base + __shfl_sync(FULL, eq_before, i) + __popc(eb & below);
-        const bool win = valid && (x > T || (x == T && rank < take_eq));
-        const uint32_t wb = __ballot_sync(FULL, win);
-        const uint32_t pos = win_base + __shfl_sync(FULL, win_before, i) + __popc(wb & below);
-        if (win) {
-          if (pos < static_cast<uint32_t>(passing))
-            out[pos] = lo + ii * NT + wt;
-          else
-            atomicOr(err_word, kErrBadIndex);
-        }
-      }
-    }
-    eq_base += tot_eq;
-    win_base += tot_win;
-  }
-}
 
 // Gather task: passing rows [c task_rows, ...) of unit u (host h, KV head g), K and V,
 // 16 bytes per thread; each thread first reads its rows' indices, then keeps eight
@@ -648,10 +440,11 @@ __global__ void __launch_bounds__(512, 1)
         const int b0 = __ldg(p.off + h), lo = b0 + (h == 0 ? p.anchor : 0), n = __ldg(p.off + h + 1) - lo;
         const float* sc = p.scores + static_cast<size_t>(g) * p.n_visual + lo;
         int32_t* out = p.idx + static_cast<size_t>(arg) * p.passing;
+        const WorkerBar bar;
         if (n <= 256 * S::kSelPer)
-          ssg_select<S::kSelPer>(sc, n, lo, p.passing, out, ctl, wt, p.err_word);
+          topp_select<256, S::kSelPer>(sc, n, lo, p.passing, out, &ctl->sel, wt, bar, p.err_word);
         else
-          ssg_select<0>(sc, n, lo, p.passing, out, ctl, wt, p.err_word);
+          topp_select<256, 0>(sc, n, lo, p.passing, out, &ctl->sel, wt, bar, p.err_word);
         worker_bar();  // every index of the unit is written (ordered before the release)
         if (wt == 0) st_release_gpu(p.unit_ready + arg, 1);
       } else {
