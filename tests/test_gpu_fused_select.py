@@ -1,6 +1,6 @@
 """The prefill's one-launch scoring + selection + gather (spava_plan_set_fused_select,
-ssg_kernel.cuh) against the three-launch path (score kernel, then select + gather)
-and the fp64 oracle.
+ssg_kernel.cuh) against the two-kernel path (score kernel, then select + gather) and
+the fp64 oracle.
 
 * Scores, indices, O and lse of the two paths are bit-identical: the fused launch
   computes the same maxima and applies the same selection rule, and the attention
@@ -12,6 +12,9 @@ and the fp64 oracle.
   registers, P = 1 with an odd anchor, and P equal to whole blocks.
 * Repeated calls on one workspace give the same result (the unit counters are
   cleared by every call).
+* With the load thread told to issue nothing, every wait of the launch (MMA issuers,
+  epilogue, publisher, worker group) runs out: the call reports SPAVA_ERR_TIMEOUT and
+  the plan then runs correctly.
 """
 
 import math
@@ -25,7 +28,10 @@ from workloads import CONFIGS
 
 from .helpers import compare_attention, inputs, make_plan, score_tolerance, to_device_bf16
 
-pytestmark = pytest.mark.gpu
+# The fused launch's CTAs wait on one another (bounded, 2 s per wait); a test that ran
+# far past that would mean a wait the kernel cannot bound, so it is ended rather than
+# left to block the rest of the suite.
+pytestmark = [pytest.mark.gpu, pytest.mark.timeout(300, method="thread")]
 
 sab = pytest.importorskip("sequence_approximate_attention_b200")
 
@@ -122,3 +128,26 @@ def test_fused_selection_with_exact_ties(dup):
             seg = np.sort(sc[r, lo:int(off[h + 1])])[::-1]
             tied += int(np.sum(seg == seg[cfg.passing - 1]) > 1)
     assert tied > 0
+
+
+def test_fused_bounded_waits_report_timeout():
+    cfg = TINY.with_(n_visual=2048, n_hosts=4, hq=4, hkv=2, head_dim=64, anchor=16, passing=64, probe_r=16,
+                     n_text=5, seed=50)
+    g, f64, dev = inputs(cfg)
+    plan = make_plan(sab, cfg, g["host_sizes"])
+    plan.set_fused_select(True)
+    ws = plan.new_workspace()
+    plan.set_debug(wait_limit_ns=20_000_000, stall_producer=True)
+    sab.attn_prefill(plan, dev["q"], dev["k"], dev["v"], workspace=ws)
+    with pytest.raises(sab.SpavaError) as ei:
+        sab.check_device_error(plan, ws)
+    assert ei.value.status == 4
+    plan.set_debug(0, False)
+    idx = torch.empty(plan.idx_shape(), dtype=torch.int32, device="cuda")
+    o, lse = sab.attn_prefill(plan, dev["q"], dev["k"], dev["v"], idx_out=idx, workspace=ws)
+    sab.check_device_error(plan, ws)
+    off = orc.host_offsets(g["host_sizes"])
+    O_ref, L_ref = orc.approx_attention(f64["q"], f64["k"], f64["v"], off, cfg.anchor,
+                                        idx.cpu().numpy().astype(np.int64), 1 / math.sqrt(cfg.head_dim))
+    compare_attention(o, lse, O_ref, L_ref, "fused, after timeout")
+    plan.close()
