@@ -45,7 +45,8 @@
  *             waits inside the kernels are bounded: a wait that runs out sets an
  *             error word in the workspace and the kernel returns;
  *             spava_check_device_error() synchronises the stream, reads that word
- *             and returns SPAVA_ERR_TIMEOUT if it is set (then clears it).
+ *             and returns SPAVA_ERR_TIMEOUT (or SPAVA_ERR_DEVICE_CHECK for a failed
+ *             range check) if it is set, then clears it.
  */
 #ifndef SPAVA_H_
 #define SPAVA_H_
@@ -62,7 +63,9 @@ typedef enum {
   SPAVA_ERR_INVALID_ARG = 1,  /* bad size, pointer, alignment or combination */
   SPAVA_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels handle    */
   SPAVA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed            */
-  SPAVA_ERR_TIMEOUT = 4       /* a bounded device wait ran out                */
+  SPAVA_ERR_TIMEOUT = 4,      /* a bounded device wait ran out                */
+  SPAVA_ERR_DEVICE_CHECK = 5  /* a device-side range check failed; the access
+                                 it guarded was skipped (none faulted)         */
 } spava_status;
 
 /* Flags of spava_score_select. */
@@ -407,7 +410,10 @@ spava_status spava_shard_stage(const spava_plan* plan, int32_t stage, const void
                                const void* v, void* o, float* lse, void* ws, void* stream);
 
 /* Synchronise `stream`, read the workspace error word, clear it.  Returns SPAVA_OK,
- * SPAVA_ERR_TIMEOUT (a bounded device wait ran out) or SPAVA_ERR_CUDA. */
+ * SPAVA_ERR_TIMEOUT (a bounded device wait ran out), SPAVA_ERR_DEVICE_CHECK (a
+ * selection position or gather index of the one-launch score/select/gather form fell
+ * outside its range and was skipped; the passing K/V are then incomplete) or
+ * SPAVA_ERR_CUDA; spava_last_error() names the error bits. */
 spava_status spava_check_device_error(const spava_plan* plan, void* ws, void* stream);
 
 /* Testing aid: the next kernel launches of this plan use a device wait limit of

@@ -14,6 +14,7 @@ SPAVA_ERR_INVALID_ARG = 1
 SPAVA_ERR_UNSUPPORTED = 2
 SPAVA_ERR_CUDA = 3
 SPAVA_ERR_TIMEOUT = 4
+SPAVA_ERR_DEVICE_CHECK = 5
 SPAVA_SCORES_GIVEN = 1
 
 SPAVA_SHARD_CONTIGUOUS = 0
@@ -95,7 +96,7 @@ class SpavaError(RuntimeError):
 
 def _status_name(s: int) -> str:
     return {0: "SPAVA_OK", 1: "SPAVA_ERR_INVALID_ARG", 2: "SPAVA_ERR_UNSUPPORTED",
-            3: "SPAVA_ERR_CUDA", 4: "SPAVA_ERR_TIMEOUT"}.get(s, f"status {s}")
+            3: "SPAVA_ERR_CUDA", 4: "SPAVA_ERR_TIMEOUT", 5: "SPAVA_ERR_DEVICE_CHECK"}.get(s, f"status {s}")
 
 
 def load(build_if_missing: bool = True):

@@ -868,6 +868,7 @@ const char* spava_status_string(spava_status s) {
     case SPAVA_ERR_UNSUPPORTED: return "SPAVA_ERR_UNSUPPORTED";
     case SPAVA_ERR_CUDA: return "SPAVA_ERR_CUDA";
     case SPAVA_ERR_TIMEOUT: return "SPAVA_ERR_TIMEOUT";
+    case SPAVA_ERR_DEVICE_CHECK: return "SPAVA_ERR_DEVICE_CHECK";
   }
   return "SPAVA_ERR_UNKNOWN";
 }
@@ -1583,6 +1584,9 @@ spava_status spava_check_device_error(const spava_plan* p, void* ws, void* strea
   if (word) {
     SPAVA_CUDA(cudaMemsetAsync(err_word(p, ws), 0, 256, st));
     SPAVA_CUDA(cudaStreamSynchronize(st));
+    if (word == spava::kErrBadIndex)
+      return fail(SPAVA_ERR_DEVICE_CHECK, "an index fell outside its range; the access was skipped (error bits 0x%x)",
+                  word);
     return fail(SPAVA_ERR_TIMEOUT, "a bounded device wait ran out (error bits 0x%x)", word);
   }
   return ok();

@@ -35,6 +35,7 @@ def test_library_exports_every_symbol(lib):
 def test_status_strings(lib):
     assert lib.spava_status_string(0) == b"SPAVA_OK"
     assert lib.spava_status_string(4) == b"SPAVA_ERR_TIMEOUT"
+    assert lib.spava_status_string(5) == b"SPAVA_ERR_DEVICE_CHECK"
 
 
 def _create(lib, **kw):
