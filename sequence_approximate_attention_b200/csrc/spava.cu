@@ -621,11 +621,13 @@ int ssg_grid(const spava_plan* p, int* smem_out, int* k_stages_out, int* task_ro
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, spava::ssg_kernel<D>, S::kThreads, smem) != cudaSuccess)
     return 0;
   if (per_sm < 1 || grid > per_sm * p->num_sms) return 0;
-  // gather tasks: at most kMaxOwnTasks per CTA
+  // gather tasks: at most kMaxOwnTasks per CTA (one unit per task the coarsest split)
   const int n_units = (p->H - 1) * p->hkv;
   int task_rows = 128;
-  while (static_cast<long long>(n_units) * ceil_div(p->P, task_rows) > static_cast<long long>(S::kMaxOwnTasks) * grid)
+  while (static_cast<long long>(n_units) * ceil_div(p->P, task_rows) > static_cast<long long>(S::kMaxOwnTasks) * grid) {
+    if (task_rows >= p->P) return 0;
     task_rows *= 2;
+  }
   *smem_out = smem;
   *k_stages_out = k_stages;
   *task_rows_out = task_rows;
