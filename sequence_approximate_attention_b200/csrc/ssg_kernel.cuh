@@ -98,7 +98,7 @@ struct SsgShape {
   static constexpr int kSmemMax = 232448;  // opt-in limit per CTA on sm_100
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kMaxOwnTasks = 64;  // gather tasks per CTA (one bit each)
-  static constexpr int kSelPer = 32;       // candidate keys per worker thread kept in registers
+  static constexpr int kSelPer = 32;       // rows of 256 candidates held in registers (one key per worker thread per row)
   static constexpr int smem_bytes(int q_bufs, int q_buf_bytes, int k_stages) {
     return q_bufs * q_buf_bytes + k_stages * kKTileBytes + kBarBytes + kItemBytes + kCtlBytes + 1024;
   }
