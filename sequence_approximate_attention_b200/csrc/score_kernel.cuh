@@ -18,9 +18,10 @@
 // of Rc probe tokens (Rc G <= 256).  Work item = one 128-key tile of one (host, KV
 // head).
 //
-// CTA = 256 threads: warp 0 TMA (one thread), warp 1 MMA (one thread), warp 2 TMEM
-// allocator, warps 4-7 epilogue (lane = key).  TMEM holds two 256-column accumulators so the
-// epilogue of one chunk overlaps the MMA of the next.
+// CTA = 256 threads: warp 0 TMA (one thread), warps 1 and 3 the two MMA issuers (one
+// thread each, one accumulator each), warp 2 TMEM allocator, warps 4-7 epilogue
+// (lane = key).  TMEM holds the two 256-column accumulators, so the epilogue of one
+// chunk overlaps the MMAs of the next.
 #pragma once
 
 #include "common.cuh"
